@@ -1,0 +1,423 @@
+#!/usr/bin/env python
+"""Benchmark of the QSA decode step on B200: queries/s and HBM roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload long|quarter|...]
+    python bench.py --impl reference ...   # the CPU oracle, timed on the host
+
+One step = one pass of the whole hot path over one batch: qsa_append_kv of the
+batch's new tokens (the current token of every sequence), qsa_index_scores,
+qsa_topk_blocks, qsa_sparse_decode, qsa_combine, all enqueued on one stream
+with the cache resident in HBM.  Between timed steps the open micro-block sums
+are restored (the step appends the same token again) and L2 is flushed by
+writing a 512 MiB buffer; neither is inside the timed events.
+
+Multi-GPU (torchrun, one rank per GPU): every rank decodes its own copy of the
+workload (independent queries; weak scaling, no data-path collective); the
+step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import configs as C  # noqa: E402
+
+METRIC = "QSA decode queries/s and HBM GB/s (% of ~8 TB/s) at 128K-256K ctx, top-512"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default="long", choices=list(C.ALL))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time budget for the CPU baseline")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+
+def dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, ws, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_close(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "200"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- algorithmic bytes
+
+
+def algorithmic_bytes(wl: C.Workload, count: np.ndarray, q_pos: np.ndarray, splits_used: int) -> dict:
+    """Bytes each kernel must move at minimum, per launch (one step)."""
+    nb = (q_pos.astype(np.int64) + 1) // 4
+    t = (q_pos.astype(np.int64) + 1) % 4
+    n_new = wl.batch * wl.new_tokens
+    tok_kv = wl.hkv * 256 * 2 * 2                       # K + V bytes of one token
+    append = n_new * (2 * tok_kv + 128 * 2)            # read new K/V/kidx, write K/V (+kc, small)
+    side = int(nb.sum()) * 128 * 2                      # kc rows read
+    scores_w = int(nb.sum()) * 4
+    index = side + scores_w
+    topk = int(nb.sum()) * 4 + wl.nq * wl.k_top * 4
+    sel_tokens = int((4 * count.astype(np.int64) + t).sum())
+    kv = sel_tokens * tok_kv
+    q_bytes = wl.nq * wl.hq * 256 * 2
+    partials = splits_used * 256 * 4
+    decode = kv + q_bytes + partials
+    out = wl.nq * wl.hq * 256 * 2
+    combine = partials + out
+    return {"append_kv": append, "index_scores": index, "topk": topk, "sparse_decode": decode, "combine": combine,
+            "pipeline_spec": side + kv + out, "side_cache": side, "selected_kv": kv, "output": out}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_sha(kernel: str) -> str:
+    src = os.path.join(ROOT, "sparse_attention_decode_03_b200", "csrc", f"{kernel}.cu")
+    common = os.path.join(ROOT, "sparse_attention_decode_03_b200", "csrc", "qsa_common.cuh")
+    h = hashlib.sha256()
+    for f in (src, common):
+        if os.path.exists(f):
+            h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current source of that kernel."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(p):
+        return None
+    txt = open(p).read()
+    m_sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", txt)
+    m_t = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    if not m_sha or not m_t or m_sha.group(1) != kernel_source_sha(kernel):
+        return None
+    return float(m_t.group(1))
+
+
+# ---------------------------------------------------------------- CPU oracle (baseline / reference arm)
+
+
+def oracle_sample(wl: C.Workload, budget_s: float, max_queries: int | None = None, start_row: int = 0):
+    """Time the CPU oracle on a bounded sample of the workload's queries.
+    Inputs (regenerated rows) are prepared first and held in host memory, like
+    the GPU's resident cache; only the oracle's own work is timed."""
+    from oracle import qsa_oracle as O
+    from tests import oracle_ref as R
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([int(i.get("num_threads", 1)) for i in threadpool_info()] or [1])
+    except Exception:  # noqa: BLE001
+        cores = 1
+    done, t_oracle = 0, 0.0
+    row = start_row
+    while t_oracle < budget_s and (max_queries is None or done < max_queries) and done < wl.nq:
+        d = R.query_inputs(wl, row % wl.nq)
+        kid = R.kidx_seq(wl, d["seq"], d["p"] + 1)
+        reader = R.kv_reader(wl, d["seq"])
+        cache = {}
+
+        def rows(pos, _r=reader, _c=cache):
+            key = np.asarray(pos).tobytes()
+            if key not in _c:
+                _c[key] = _r(pos)
+            return _c[key]
+        O.decode_query(d["q"], d["q_idx"], d["w"], d["p"], kid, rows, wl.k_top, wl.scale)   # untimed: fetch rows
+        t0 = time.perf_counter()
+        O.decode_query(d["q"], d["q_idx"], d["w"], d["p"], kid, rows, wl.k_top, wl.scale)
+        t_oracle += time.perf_counter() - t0
+        done += 1
+        row += max(1, wl.nq // 7)
+    return done, t_oracle, cores
+
+
+def run_reference(args, rank, ws):
+    if rank != 0:
+        return
+    wl = C.get(args.workload)
+    per_step = []
+    total_q = 0
+    budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        n, t, cores = oracle_sample(wl, budget, max_queries=2, start_row=i)
+        if i >= args.warmup:
+            per_step.append(t / n)
+            total_q += n
+    qps = 1.0 / statistics.mean(per_step)
+    line = {"impl": "reference", "metric": METRIC, "value": qps, "unit": "queries/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * statistics.mean(per_step) * wl.nq,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {**wl.describe(), "parallelism": "host cores"},
+            "cpu_baseline": {"value": qps, "unit": "queries/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{total_q} queries of the workload, fp64 numpy oracle, inputs regenerated "
+                                       f"and resident in host memory"},
+            "e2e": {"value": qps, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- native arm
+
+
+def run_native(args, rank, ws, local):
+    import sparse_attention_decode_03_b200 as qsa
+    from workloads import harness as H
+
+    wl = C.get(args.workload)
+    dev = torch.device("cuda", local)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    cache = H.build_cache(wl, dev_status=st)
+    inp = H.step_inputs(wl)
+    dec = qsa.Decoder(cache, wl.hq, wl.nq, k=wl.k_top, scale=wl.scale, target_ctas=sms,
+                      chunk_units=H.chunk_units_for(wl))
+    dec.dev_status = st
+    saved_partial = cache.kc_partial.clone()
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    names = ["append_kv", "index_scores", "topk", "sparse_decode", "combine"]
+
+    def step(evs=None):
+        if evs:
+            evs[0].record()
+        qsa.qsa_append_kv(cache, inp["k_new"], inp["v_new"], inp["kidx_new"], inp["seq_id"], inp["pos"], st)
+        if evs:
+            evs[1].record()
+        nq = wl.nq
+        qsa.qsa_index_scores(cache, inp["q_idx"], inp["w"], inp["q_seq"], inp["q_pos"], dec.scores[:nq], st)
+        if evs:
+            evs[2].record()
+        qsa.qsa_topk_blocks(dec.scores[:nq], inp["q_pos"], wl.k_top, dec.sel[:nq], dec.count[:nq], st)
+        if evs:
+            evs[3].record()
+        qsa.qsa_sparse_decode(cache, inp["q"], inp["q_seq"], inp["q_pos"], dec.sel[:nq], dec.count[:nq], wl.k_top,
+                              wl.scale, dec.chunk_units, dec.max_splits, dec.part_o[:nq], dec.part_lse[:nq], st)
+        if evs:
+            evs[4].record()
+        qsa.qsa_combine(dec.part_o[:nq], dec.part_lse[:nq], dec.out[:nq], dec.lse[:nq])
+        if evs:
+            evs[5].record()
+
+    def between():
+        cache.kc_partial.copy_(saved_partial)
+        flush.zero_()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+        between()
+    torch.cuda.synchronize()
+    status = int(st.item())
+    if status:
+        raise RuntimeError(f"device status {qsa.dev_status_names(status)}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        wall0 = time.perf_counter()
+        for i in range(args.steps):
+            step(evs[i])
+            between()
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - wall0
+    barrier(ws)
+    step_ms = [evs[i][0].elapsed_time(evs[i][5]) for i in range(args.steps)]
+    kern_ms = {n: statistics.mean(evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(args.steps))
+               for k, n in enumerate(names)}
+    mean_ms = statistics.mean(step_ms)
+    total_ms = max_over_ranks(sum(step_ms), ws)
+    value = ws * wl.nq * args.steps / (total_ms / 1000.0)
+
+    # ---- e2e: public API with pinned host buffers, H2D + step + D2H inside the timed events
+    keys = ["k_new", "v_new", "kidx_new", "seq_id", "pos", "q", "q_idx", "w", "q_seq", "q_pos"]
+    host = {k: inp[k].cpu().pin_memory() for k in keys}
+    out_h = torch.empty(dec.out[:wl.nq].shape, dtype=dec.out.dtype).pin_memory()
+    lse_h = torch.empty(dec.lse[:wl.nq].shape, dtype=dec.lse.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+    e2e_ms = []
+    for i in range(args.steps + 2):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for k in keys:
+            inp[k].copy_(host[k], non_blocking=True)
+        step()
+        out_h.copy_(dec.out[:wl.nq], non_blocking=True)
+        lse_h.copy_(dec.lse[:wl.nq], non_blocking=True)
+        e1.record()
+        e1.synchronize()
+        if i >= 2:
+            e2e_ms.append(e0.elapsed_time(e1))
+        between()
+    torch.cuda.synchronize()
+    e2e_total = max_over_ranks(sum(e2e_ms), ws)
+    e2e_value = ws * wl.nq * len(e2e_ms) / (e2e_total / 1000.0)
+
+    # ---- roofline of the dominant kernel
+    count = dec.count[:wl.nq].cpu().numpy()
+    q_pos = inp["q_pos"].cpu().numpy()
+    n_slots = wl.nq * wl.hkv * (wl.k_top + 1)
+    chunks = math.ceil(n_slots / dec.chunk_units)
+    splits_used = (chunks + wl.nq * wl.hkv) * (wl.hq // wl.hkv)
+    ab = algorithmic_bytes(wl, count, q_pos, splits_used)
+    peak, peak_kind = measured_peaks()
+    dom = max(names, key=lambda n: kern_ms[n])
+    dom_key = {"topk": "topk"}.get(dom, dom)
+    achieved = ab[dom_key] / (kern_ms[dom] / 1000.0) / 1e9
+    traffic = profiled_traffic(dom, args.workload)
+    kernels = {n: {"ms": round(kern_ms[n], 5), "alg_bytes": ab[n],
+                   "gbs": round(ab[n] / (kern_ms[n] / 1000.0) / 1e9, 1)} for n in names}
+    pipeline_gbs = ab["pipeline_spec"] / (mean_ms / 1000.0) / 1e9
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": mean_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {**wl.describe(), "l2": "flushed (512 MiB write) between timed steps",
+                   "step": "append_kv + index_scores + topk_blocks + sparse_decode + combine",
+                   "parallelism": f"dp{ws} (independent replicas)" if ws > 1 else "single GPU",
+                   "chunk_units": dec.chunk_units, "max_splits": dec.max_splits},
+        "hbm": {"pipeline_alg_bytes": ab["pipeline_spec"], "achieved_gbs": round(pipeline_gbs, 1), "peak_gbs": peak,
+                "frac": round(pipeline_gbs / peak, 4), "peak_kind": f"{peak_kind} STREAM copy"},
+        "roofline": {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "alg_bytes_per_launch": ab[dom_key], "peak_kind": f"{peak_kind} (hbm_gbs)"},
+        "kernels": kernels,
+        "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": statistics.mean(e2e_ms)},
+        "gpu_launches": 6 * args.steps,
+        "clocks": clk.summary(),
+        "wall_s_timed_region": round(wall, 3),
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        n, t, cores = oracle_sample(wl, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": n / t, "unit": "queries/s", "cores": cores, "kind": "oracle",
+                                "sample": f"{n} of the workload's {wl.nq} queries (rows spread over the batch), "
+                                          f"fp64 numpy oracle, inputs regenerated and resident in host memory"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    rank, ws, local = dist_init()
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, ws)
+        else:
+            run_native(args, rank, ws, local)
+    finally:
+        dist_close(ws)
+
+
+if __name__ == "__main__":
+    main()

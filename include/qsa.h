@@ -1,0 +1,221 @@
+/*
+ * qsa.h -- C ABI of libqsa: the Qwen Sparse Attention (QSA) decode hot path on
+ * one NVIDIA B200 (sm_100a).
+ *
+ * What the path computes (sources: the pages
+ *   [DCP]  "Qwen 4 QSA krijgt decode-contextparallellisme: in vLLM's concept-PR
+ *          voor Qwen3.8-Flash-Next", section "Wat de pull request daadwerkelijk
+ *          verandert";
+ *   [CANN] "Qwen4-Exp QSA komt naar Huawei's Ascend: binnen SGLang's opt-in CANN
+ *          prefill-PR", sections "Wat de pull request daadwerkelijk toevoegt",
+ *          "Negen tests die geslaagd zijn ..." and "Waarom QSA het lastige
+ *          onderdeel is, in cijfers";
+ *   [BSS]  "Pengambilan sampel batch-sharded Qwen4Exp", section "Apa yang
+ *          dikatakan oleh klaster patch di sekitarnya tentang Qwen4Exp"):
+ *   a lightweight indexer compresses keys into micro-blocks of 4 tokens and
+ *   scores every block against the query; the best 512 blocks (about 2,048
+ *   token positions) are kept; softmax and value aggregation then run over the
+ *   uncompressed BF16 K and V (head dim 256, GQA) at those positions only; the
+ *   attention is split over KV chunks and merged with log-sum-exp (the
+ *   single-GPU analogue of the cross-rank combine of [DCP]).
+ * Fixed readings where the pages are silent: kc_j = sum of the 4 tokens'
+ * indexer keys (fp32, token order, stored BF16 round-to-nearest-even);
+ * s_j = sum_h w_h * ReLU(q_idx,h . kc_j) with 8 indexer heads of dim 128; ties
+ * go to the lower block index; a query at position p sees nb = (p+1)/4
+ * complete blocks and always attends its t = (p+1)%4 trailing tokens.
+ *
+ * Conventions for every call
+ *  - Pointers are DEVICE pointers owned and allocated by the caller, except
+ *    the `cache` descriptor itself (host memory, read during the call only).
+ *    The library allocates nothing and never synchronises the host.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream); calls only
+ *    enqueue work on it.
+ *  - Return value: QSA_OK, or a negative qsa_status for a host-detected error
+ *    (nothing is enqueued then).
+ *  - `dev_status` (may be NULL) is a device int32 the kernels OR error bits
+ *    into (QSA_DEV_*) when they meet bad data: an out-of-range page id,
+ *    sequence id, position, selection index or count.  The offending read is
+ *    skipped (masked); kernels never trap.  The caller clears and reads it.
+ *  - All outputs are deterministic: no floating-point atomics.
+ *  - Tensors are dense row-major with the shapes given; no strides.
+ */
+#ifndef QSA_H
+#define QSA_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QSA_API __attribute__((visibility("default")))
+#else
+#define QSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* fixed geometry ([CANN] "Waarom QSA ...": head dim 256, indexer dim 128,
+ * ratio 4; indexer heads 8 and 64-token pages are fixed readings) */
+#define QSA_HEAD_DIM 256
+#define QSA_IDX_HEADS 8
+#define QSA_IDX_DIM 128
+#define QSA_RATIO 4
+#define QSA_PAGE_TOKENS 64
+#define QSA_BLOCKS_PER_PAGE 16 /* micro-blocks per page */
+#define QSA_MAX_TOPK 2048      /* largest K accepted by qsa_topk_blocks / qsa_sparse_decode */
+#define QSA_MAX_GROUP 16       /* largest Hq / Hkv accepted by qsa_sparse_decode */
+
+typedef enum {
+  QSA_OK = 0,
+  QSA_ERR_INVALID_ARG = -1, /* null pointer, negative size, Hq % Hkv != 0, K > QSA_MAX_TOPK, ... */
+  QSA_ERR_UNSUPPORTED = -2, /* a shape the kernels do not implement (e.g. Hq / Hkv > 16) */
+  QSA_ERR_CUDA = -3         /* a CUDA launch failed; cudaGetLastError() has been cleared */
+} qsa_status;
+
+/* bits OR-ed into *dev_status by the kernels */
+#define QSA_DEV_BAD_PAGE 1    /* block-table entry outside [0, num_pages) */
+#define QSA_DEV_BAD_SEQ 2     /* sequence id outside [0, max_seqs) */
+#define QSA_DEV_BAD_POS 4     /* position < 0 or beyond the block-table capacity */
+#define QSA_DEV_BAD_SEL 8     /* selected block index outside [0, nb_q) */
+#define QSA_DEV_BAD_COUNT 16  /* selection count outside [0, min(K, nb_q)] */
+#define QSA_DEV_BAD_ORDER 32  /* append tokens of one sequence not in consecutive positions */
+#define QSA_DEV_TIMEOUT 64    /* a bounded pipeline wait expired; outputs of that call are invalid */
+#define QSA_DEV_SCORES_LD 128 /* a query sees more blocks than the scores row holds */
+
+/*
+ * One cache group ([DCP]: the selector and the main KV cache are kept in one
+ * cache group so they cannot drift apart).  The main K/V and the compressed
+ * indexer side cache are paged by the SAME physical page ids.
+ *   k_pages, v_pages  bf16 [num_pages][num_kv_heads][64][256]  post-RoPE K / V
+ *   kc_pages          bf16 [num_pages][16][128]  kc of the 16 micro-blocks of a page
+ *   kc_partial        fp32 [max_seqs][128]       running fp32 sum of each sequence's
+ *                                                 open (incomplete) micro-block
+ *   block_table       int32 [max_seqs][max_pages_per_seq]  logical page -> physical page
+ * All buffers are caller-owned device memory; the library writes k/v/kc pages
+ * and kc_partial only in qsa_append_kv.
+ */
+typedef struct {
+  void* k_pages;
+  void* v_pages;
+  void* kc_pages;
+  float* kc_partial;
+  const int32_t* block_table;
+  int32_t num_pages;
+  int32_t max_seqs;
+  int32_t max_pages_per_seq;
+  int32_t num_kv_heads;
+} qsa_cache_t;
+
+/* Human-readable name of a qsa_status value (static string). */
+QSA_API const char* qsa_status_string(int status);
+
+/* ABI version of this header (bumped on any signature change). */
+QSA_API int qsa_abi_version(void);
+#define QSA_ABI_VERSION 1
+
+/*
+ * qsa_append_kv -- write n new tokens into the cache group.
+ * [DCP] keeps the selector caches in step with the main cache; [CANN] marks
+ * invalid slots with -1 padding and [DCP] stops synthetic batches from writing
+ * the QSA side caches: a token with seq_id < 0 is skipped entirely.
+ *   k_new, v_new  bf16 [n][Hkv][256];  kidx_new  bf16 [n][128] (indexer keys)
+ *   seq_id, pos   int32 [n]  sequence and absolute position of each token
+ * Effect: K/V rows written at page block_table[seq][pos/64], row pos%64.  The
+ * indexer keys of a micro-block are summed in fp32 in token order (continuing
+ * kc_partial when the block began in an earlier call); when the token at
+ * position 4j+3 arrives, kc_pages row j = BF16(sum) (round to nearest even).
+ * A block left incomplete stores its running sum in kc_partial[seq].
+ * Rules: the tokens of one sequence are contiguous in the arrays and at
+ * consecutive increasing positions, and calls for a sequence arrive in
+ * position order (violations set QSA_DEV_BAD_ORDER).  Two kernels are
+ * enqueued.  n = 0 is a no-op.
+ */
+QSA_API int qsa_append_kv(const qsa_cache_t* cache, const void* k_new, const void* v_new, const void* kidx_new,
+                  const int32_t* seq_id, const int32_t* pos, int32_t n, int32_t* dev_status, void* stream);
+
+/*
+ * qsa_index_scores -- [DCP]/[CANN]/[BSS]: the indexer scores every complete
+ * micro-block visible to each query:
+ *   scores[q][j] = sum_{h<8} w[q][h] * max(0, sum_{d<128} q_idx[q][h][d] * kc[seq_q][j][d])
+ * for j < nb_q = (q_pos[q] + 1) / 4 (entries j >= nb_q are not written).
+ *   q_idx bf16 [nq][8][128]; w fp32 [nq][8]; q_seq, q_pos int32 [nq]
+ *   scores fp32 [nq][scores_ld]; scores_ld >= the largest nb_q
+ * Products are BF16 x BF16 accumulated in fp32 on the tensor cores; with
+ * integer-valued indexer data and power-of-two weights every score is exact.
+ * A page-table miss writes -inf for its 16 blocks and sets QSA_DEV_BAD_PAGE.
+ */
+QSA_API int qsa_index_scores(const qsa_cache_t* cache, const void* q_idx, const float* w, const int32_t* q_seq,
+                     const int32_t* q_pos, int32_t nq, float* scores, int64_t scores_ld, int32_t* dev_status,
+                     void* stream);
+
+/*
+ * qsa_topk_blocks -- per query, keep the best min(k, nb_q) blocks ([DCP]: "the
+ * best 512 blocks") under the order (score descending, block index
+ * ascending), written sorted by block index ascending:
+ *   sel   int32 [nq][k]  selected block indices, then -1 padding
+ *   count int32 [nq]     min(k, nb_q)
+ * Deterministic radix select on the fp32 bit patterns; 0 <= k <= QSA_MAX_TOPK.
+ */
+QSA_API int qsa_topk_blocks(const float* scores, int64_t scores_ld, const int32_t* q_pos, int32_t nq, int32_t k,
+                    int32_t* sel, int32_t* count, int32_t* dev_status, void* stream);
+
+/*
+ * qsa_decode_plan -- host-only helper: choose the KV chunk size for
+ * qsa_sparse_decode.  Every (query, KV head) pair owns k+1 unit slots (its k
+ * selection slots, then its trailing micro-block); the slots of all pairs,
+ * query-major, are cut into chunks of *chunk_units slots, one CTA per chunk.
+ * The chunk size spreads the nq*hkv*(k+1) slots over about target_ctas CTAs
+ * (pass the SM count).  *max_splits = the most chunks one pair can touch,
+ * i.e. the split dimension S of part_o / part_lse.
+ */
+QSA_API int qsa_decode_plan(int32_t nq, int32_t hkv, int32_t k, int32_t target_ctas, int32_t* chunk_units,
+                    int32_t* max_splits);
+
+/*
+ * qsa_sparse_decode -- sparse attention over the uncompressed K/V at the
+ * selected positions ([DCP]: softmax and value aggregation run on the
+ * uncompressed K and V), split over KV chunks ([DCP]: split read, results
+ * combined afterwards).
+ * For query q (position p, nb = (p+1)/4, t = (p+1)%4) and KV head g, unit slot
+ * u < count[q] holds the 4 tokens of block sel[q][u]; slots count[q]..k-1 are
+ * empty; slot k holds the t trailing tokens 4nb..p.  Chunk c covers the global
+ * slots [c*chunk_units, (c+1)*chunk_units) of the order (q, g, u); the part of
+ * pair (q, g) inside the s-th chunk it touches is split s.  For every Q head h
+ * of group g (h / (hq/hkv) == g) and split s over token set T:
+ *   z_t = scale * q[q][h] . K[t][g];  lse = log sum_t exp(z_t);
+ *   o = sum_t exp(z_t - lse) V[t][g]
+ * written to part_o[q][s][h][:] (fp32) and part_lse[q][s][h] (fp32, natural
+ * log).  An empty split, and every slot s a pair does not reach, gets o = 0
+ * and lse = -inf ([CANN]: fully masked rows keep the zero-output convention).
+ *   q bf16 [nq][hq][256]; sel int32 [nq][k]; count int32 [nq]
+ *   part_o fp32 [nq][max_splits][hq][256]; part_lse fp32 [nq][max_splits][hq]
+ * Requirements: hq % Hkv == 0, hq / Hkv <= 16, 0 <= k <= QSA_MAX_TOPK,
+ * chunk_units >= 1, max_splits >= the value qsa_decode_plan reports for
+ * (k, chunk_units), scale > 0 (the pages keep the D256 scale 1/16).
+ * The kernel gathers each selected micro-block (4 tokens x 512 B of K and of V
+ * per KV head, contiguous in a page) with bulk async copies into shared memory
+ * and runs QK^T and PV on the tensor cores with fp32 accumulation; P is
+ * rounded to BF16 for PV.
+ */
+QSA_API int qsa_sparse_decode(const qsa_cache_t* cache, const void* q, int32_t nq, int32_t hq, const int32_t* q_seq,
+                      const int32_t* q_pos, const int32_t* sel, const int32_t* count, int32_t k, float scale,
+                      int32_t chunk_units, int32_t max_splits, float* part_o, float* part_lse,
+                      int32_t* dev_status, void* stream);
+
+/*
+ * qsa_combine -- log-sum-exp merge of the splits ([DCP]: attention results of
+ * the split read are combined):
+ *   lse[q][h] = log sum_s exp(part_lse[q][s][h]);
+ *   out[q][h] = BF16( sum_s exp(part_lse[q][s][h] - lse[q][h]) * part_o[q][s][h] )
+ * Splits with lse = -inf are skipped; if all are, out = 0 exactly and
+ * lse = -inf ([CANN] zero-output convention).
+ *   out bf16 [nq][hq][256]; lse fp32 [nq][hq]
+ */
+QSA_API int qsa_combine(const float* part_o, const float* part_lse, int32_t nq, int32_t max_splits, int32_t hq,
+                void* out, float* lse, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QSA_H */

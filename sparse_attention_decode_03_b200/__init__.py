@@ -1,0 +1,9 @@
+"""QSA (Qwen Sparse Attention) decode hot path for one NVIDIA B200 (sm_100a).
+
+The compute runs in libqsa.so (hand-written CUDA, C ABI in include/qsa.h); this
+package is its thin ctypes binding.  Build the library with
+``python -m sparse_attention_decode_03_b200.build``.
+"""
+from .qsa import (  # noqa: F401
+    ABI_VERSION, LIB_PATH, Decoder, PagedCache, QSAError, dev_status_names, qsa_append_kv, qsa_combine,
+    qsa_decode_plan, qsa_index_scores, qsa_sparse_decode, qsa_topk_blocks, splits_bound, status_string)

@@ -1,0 +1,155 @@
+// qsa_append_kv: scatter new tokens into the paged cache group and maintain the
+// compressed indexer side cache (kc = fp32 sum of a micro-block's 4 indexer keys,
+// stored BF16), continuing a block across calls through kc_partial.
+//
+// Source: [DCP] "Qwen 4 QSA krijgt decode-contextparallellisme ...", section
+// "Wat de pull request daadwerkelijk verandert" (indexer compresses keys into
+// micro-blocks of ratio 4; selector and main KV in one cache group; synthetic
+// batches do not write the side caches) and [CANN] "Qwen4-Exp QSA komt naar
+// Huawei's Ascend ...", section "Wat de pull request daadwerkelijk toevoegt"
+// (-1 padding marks slots that must not be used).
+//
+// Two kernels, one warp per token:
+//   scatter: writes K/V rows; the token at position 4j+3 closes block j and
+//            writes kc row j (partial of earlier calls + this call's tokens);
+//   partial: the last token of a sequence's run, if its block is still open,
+//            writes the running sum to kc_partial.
+// Splitting the partial write into a second launch orders it after every read
+// of the old partial in the first one.
+#include "qsa_common.cuh"
+
+namespace {
+
+using namespace qsa;
+
+constexpr int kWarps = 8;
+
+struct AppendArgs {
+  qsa_cache_t c;
+  const __nv_bfloat16* k_new;
+  const __nv_bfloat16* v_new;
+  const __nv_bfloat16* kidx;
+  const int32_t* seq_id;
+  const int32_t* pos;
+  int32_t n;
+  int32_t* st;
+};
+
+// Number of this call's tokens directly before `tok` that belong to the same
+// sequence at consecutive positions (at most `limit`).
+__device__ __forceinline__ int run_before(const AppendArgs& a, int64_t tok, int seq, int p, int limit) {
+  int m = 0;
+  while (m < limit && tok - m - 1 >= 0 && a.seq_id[tok - m - 1] == seq && a.pos[tok - m - 1] == p - m - 1) ++m;
+  return m;
+}
+
+// fp32 running sum (4 dims per lane) of tokens tok-m .. tok, starting from
+// kc_partial[seq] when the block began before this call.
+__device__ __forceinline__ float4 block_sum(const AppendArgs& a, int64_t tok, int seq, int m, bool from_partial,
+                                            int lane) {
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (from_partial) acc = *reinterpret_cast<const float4*>(a.c.kc_partial + (size_t)seq * kIdxDim + lane * 4);
+  for (int i = m; i >= 0; --i) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(a.kidx + (size_t)(tok - i) * kIdxDim + lane * 4);
+    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+    acc.x = __fadd_rn(acc.x, lo.x);
+    acc.y = __fadd_rn(acc.y, lo.y);
+    acc.z = __fadd_rn(acc.z, hi.x);
+    acc.w = __fadd_rn(acc.w, hi.y);
+  }
+  return acc;
+}
+
+__global__ void __launch_bounds__(kWarps * 32) append_scatter_kernel(AppendArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t tok = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  if (tok >= a.n) return;
+  const int seq = a.seq_id[tok];
+  if (seq < 0) return;  // padding / synthetic token: writes nothing
+  const int p = a.pos[tok];
+  if (seq >= a.c.max_seqs) {
+    if (lane == 0) flag(a.st, QSA_DEV_BAD_SEQ);
+    return;
+  }
+  if (p < 0 || (int64_t)p >= (int64_t)a.c.max_pages_per_seq * kPage) {
+    if (lane == 0) flag(a.st, QSA_DEV_BAD_POS);
+    return;
+  }
+  if (lane == 0 && tok > 0 && a.seq_id[tok - 1] == seq && a.pos[tok - 1] != p - 1) flag(a.st, QSA_DEV_BAD_ORDER);
+  const int page = a.c.block_table[(int64_t)seq * a.c.max_pages_per_seq + p / kPage];
+  if (page < 0 || page >= a.c.num_pages) {
+    if (lane == 0) flag(a.st, QSA_DEV_BAD_PAGE);
+    return;
+  }
+  const int slot = p % kPage;
+  const int hkv = a.c.num_kv_heads;
+  __nv_bfloat16* kp = static_cast<__nv_bfloat16*>(a.c.k_pages);
+  __nv_bfloat16* vp = static_cast<__nv_bfloat16*>(a.c.v_pages);
+  for (int h = 0; h < hkv; ++h) {
+    const size_t dst = (((size_t)page * hkv + h) * kPage + slot) * kHeadDim + lane * 8;
+    const size_t src = ((size_t)tok * hkv + h) * kHeadDim + lane * 8;
+    *reinterpret_cast<uint4*>(kp + dst) = *reinterpret_cast<const uint4*>(a.k_new + src);
+    *reinterpret_cast<uint4*>(vp + dst) = *reinterpret_cast<const uint4*>(a.v_new + src);
+  }
+  if ((p & 3) == 3) {  // this token closes micro-block p / 4
+    const int m = run_before(a, tok, seq, p, 3);
+    const float4 acc = block_sum(a, tok, seq, m, m < 3, lane);
+    __nv_bfloat16* kc = static_cast<__nv_bfloat16*>(a.c.kc_pages) +
+                        ((size_t)page * kBlocksPerPage + slot / kRatio) * kIdxDim + lane * 4;
+    uint2 out;
+    out.x = pack_bf16(acc.x, acc.y);
+    out.y = pack_bf16(acc.z, acc.w);
+    *reinterpret_cast<uint2*>(kc) = out;
+  }
+}
+
+__global__ void __launch_bounds__(kWarps * 32) append_partial_kernel(AppendArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t tok = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  if (tok >= a.n) return;
+  const int seq = a.seq_id[tok];
+  if (seq < 0 || seq >= a.c.max_seqs) return;
+  const int p = a.pos[tok];
+  if (p < 0 || (int64_t)p >= (int64_t)a.c.max_pages_per_seq * kPage) return;
+  const int r = p & 3;
+  if (r == 3) return;  // block closed by this token: nothing left open
+  const bool last = (tok == a.n - 1) || a.seq_id[tok + 1] != seq || a.pos[tok + 1] != p + 1;
+  if (!last) return;
+  const int m = run_before(a, tok, seq, p, r);
+  const float4 acc = block_sum(a, tok, seq, m, m < r, lane);
+  *reinterpret_cast<float4*>(a.c.kc_partial + (size_t)seq * kIdxDim + lane * 4) = acc;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" int qsa_append_kv(const qsa_cache_t* cache, const void* k_new, const void* v_new, const void* kidx_new,
+                             const int32_t* seq_id, const int32_t* pos, int32_t n, int32_t* dev_status,
+                             void* stream) {
+  if (!cache || n < 0) return QSA_ERR_INVALID_ARG;
+  if (n == 0) return QSA_OK;
+  const qsa_cache_t& c = *cache;
+  if (!c.k_pages || !c.v_pages || !c.kc_pages || !c.kc_partial || !c.block_table) return QSA_ERR_INVALID_ARG;
+  if (!k_new || !v_new || !kidx_new || !seq_id || !pos) return QSA_ERR_INVALID_ARG;
+  if (c.num_pages < 1 || c.max_seqs < 1 || c.max_pages_per_seq < 1 || c.num_kv_heads < 1) return QSA_ERR_INVALID_ARG;
+  if (!aligned16(c.k_pages) || !aligned16(c.v_pages) || !aligned16(c.kc_partial) || !aligned16(k_new) ||
+      !aligned16(v_new) || (reinterpret_cast<uintptr_t>(c.kc_pages) & 7u) || (reinterpret_cast<uintptr_t>(kidx_new) & 7u))
+    return QSA_ERR_INVALID_ARG;
+  AppendArgs a{c,
+               static_cast<const __nv_bfloat16*>(k_new),
+               static_cast<const __nv_bfloat16*>(v_new),
+               static_cast<const __nv_bfloat16*>(kidx_new),
+               seq_id,
+               pos,
+               n,
+               dev_status};
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned grid = (unsigned)((n + kWarps - 1) / kWarps);
+  append_scatter_kernel<<<grid, kWarps * 32, 0, s>>>(a);
+  int rc = qsa_host::launch_status();
+  if (rc != QSA_OK) return rc;
+  append_partial_kernel<<<grid, kWarps * 32, 0, s>>>(a);
+  return qsa_host::launch_status();
+}

@@ -1,0 +1,552 @@
+// qsa_sparse_decode: softmax attention of every Q head over the selected
+// micro-blocks (plus the causal tail) of its query, on the uncompressed BF16
+// K/V, written as split-KV partials (o, lse).
+//
+// Source: [DCP] "Qwen 4 QSA krijgt decode-contextparallellisme ...", section
+// "Wat de pull request daadwerkelijk verandert" (final softmax and value
+// aggregation on the uncompressed K and V; the split read is combined
+// afterwards); [CANN] "Qwen4-Exp QSA komt naar Huawei's Ascend ...", sections
+// "Wat de pull request daadwerkelijk toevoegt" (D256 scale, zero output for
+// fully masked rows) and "Negen tests ..." (causal tail remainders 0..3).
+//
+// Work decomposition.  Each (query, KV head) pair owns K+1 unit slots: the K
+// selection slots (one micro-block of 4 tokens each, 2 KiB of K and 2 KiB of V
+// per KV head, contiguous in a page) and the tail slot.  All slots, query
+// major, are cut into fixed chunks; one CTA per chunk, so every SM gets the
+// same number of slots whatever the batch shape.  The part of a pair inside a
+// chunk is a "segment"; each segment yields one split partial.
+//
+// CTA = 1 producer warp + 4 consumer warps, 1 CTA per SM.
+//   producer: looks up 32 units at a time (selection -> page table), then per
+//     tile of 4 units issues cp.async.bulk copies of the K and V micro-blocks
+//     into a 6-stage shared-memory ring (mbarrier full/empty pairs).
+//   consumers: each warp takes whole tiles (16 tokens) of the segment and runs
+//     S = Q K^T and O += P V with mma.sync m16n8k16 (M = 16 Q-head rows of the
+//     KV group, fp32 accumulate), online softmax in registers; at the end of a
+//     segment the 4 warps merge their (m, l, O) through shared memory and write
+//     the partial.
+// Shared-memory layouts are skewed so that every 16-byte fragment read is
+// bank-conflict free (micro-block slots 2080 B apart, Q rows 576 B apart).
+#include "qsa_common.cuh"
+
+namespace {
+
+using namespace qsa;
+
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kStages = 6;
+constexpr int kUnitsPerTile = 4;
+constexpr int kUnitBytes = kRatio * kHeadDim * 2;                      // 2048
+constexpr int kSlotStride = kUnitBytes + 32;                           // 2080
+constexpr int kStageBytes = 2 * kUnitsPerTile * kSlotStride;           // K slots then V slots
+constexpr int kQRowStride = kHeadDim * 2 + 64;                         // 576
+constexpr int kQBufBytes = 16 * kQRowStride;
+constexpr int kCombRow = kHeadDim + 4;                                 // floats
+constexpr int kCombBytes = kConsumerWarps * 16 * kCombRow * 4;
+constexpr int kOffRing = 0;
+constexpr int kOffQ = kOffRing + kStages * kStageBytes;
+constexpr int kOffComb = kOffQ + 2 * kQBufBytes;
+constexpr int kOffML = kOffComb + kCombBytes;
+constexpr int kOffMeta = kOffML + kConsumerWarps * 16 * 2 * 4;
+constexpr int kOffBar = (kOffMeta + kStages * 4 + 7) & ~7;
+constexpr int kOffAbort = kOffBar + 2 * kStages * 8;
+constexpr int kSmemBytes = kOffAbort + 16;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr int kBarConsumers = 1;                  // named barrier id
+
+struct DecodeArgs {
+  const __nv_bfloat16* k_pages;
+  const __nv_bfloat16* v_pages;
+  const int32_t* bt;
+  int32_t num_pages, max_seqs, mpps, hkv;
+  const __nv_bfloat16* q;
+  int32_t hq, G;
+  const int32_t* q_seq;
+  const int32_t* q_pos;
+  const int32_t* sel;
+  const int32_t* count;
+  int32_t K;
+  float scale_log2;
+  int64_t chunk;
+  int64_t total_slots;
+  int32_t max_splits;
+  float* part_o;
+  float* part_lse;
+  int32_t* st;
+};
+
+struct Seg {
+  int q, g, split;
+  int u0, u1;  // unit slots [u0, u1) of the pair
+  int seq, nb, t;
+  int n_main;  // selected blocks in the segment
+  int n_valid, n_tiles;
+  bool has_tail, last_of_pair, query_ok;
+};
+
+// Segment of pair `pair` inside chunk [x0, x1).  Identical in every warp.
+__device__ __forceinline__ Seg make_seg(const DecodeArgs& a, int64_t pair, int64_t x0, int64_t x1, bool report) {
+  Seg s;
+  const int64_t n_slots = (int64_t)a.K + 1;
+  const int64_t base = pair * n_slots;
+  s.q = (int)(pair / a.hkv);
+  s.g = (int)(pair % a.hkv);
+  s.split = (int)(blockIdx.x - base / a.chunk);
+  s.u0 = (int)(max(x0, base) - base);
+  s.u1 = (int)(min(x1, base + n_slots) - base);
+  s.last_of_pair = s.u1 == (int)n_slots;
+  s.seq = a.q_seq[s.q];
+  const int p = a.q_pos[s.q];
+  s.query_ok = s.seq >= 0 && s.seq < a.max_seqs && p >= 0 && (int64_t)p < (int64_t)a.mpps * kPage;
+  if (!s.query_ok) {
+    if (report) flag(a.st, (s.seq < 0 || s.seq >= a.max_seqs) ? QSA_DEV_BAD_SEQ : QSA_DEV_BAD_POS);
+    s.nb = 0;
+    s.t = 0;
+  } else {
+    s.nb = (p + 1) / kRatio;
+    s.t = (p + 1) % kRatio;
+  }
+  int cnt = s.query_ok ? a.count[s.q] : 0;
+  const int cap = min(a.K, s.nb);
+  if (cnt < 0 || cnt > cap) {
+    if (report) flag(a.st, QSA_DEV_BAD_COUNT);
+    cnt = cnt < 0 ? 0 : cap;
+  }
+  s.n_main = max(0, min(s.u1, cnt) - s.u0);
+  s.has_tail = s.u0 <= a.K && a.K < s.u1 && s.t > 0;
+  s.n_valid = s.n_main + (s.has_tail ? 1 : 0);
+  s.n_tiles = (s.n_valid + kUnitsPerTile - 1) / kUnitsPerTile;
+  return s;
+}
+
+// ------------------------------------------------------------------ producer
+
+__device__ void producer(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_t x1) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t ring = smem_u32(smem + kOffRing);
+  const uint32_t bar_full = smem_u32(smem + kOffBar);
+  const uint32_t bar_empty = bar_full + kStages * 8;
+  uint32_t* meta = reinterpret_cast<uint32_t*>(smem + kOffMeta);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
+  const uint64_t policy = l2_policy_evict_first();
+  const int64_t n_slots = (int64_t)a.K + 1;
+  int64_t T = 0;
+  bool aborted = false;
+
+  for (int64_t pair = x0 / n_slots; pair <= (x1 - 1) / n_slots && !aborted; ++pair) {
+    const Seg s = make_seg(a, pair, x0, x1, false);
+    for (int ub = 0; ub < s.n_valid && !aborted; ub += 32) {
+      // lane i describes unit ub + i of the segment
+      const int i = ub + lane;
+      uint32_t rows = 0;
+      size_t off = 0;
+      bool copy = false;
+      if (i < s.n_valid) {
+        int j, nrows;
+        bool ok = true;
+        if (i < s.n_main) {
+          j = a.sel[(size_t)s.q * a.K + s.u0 + i];
+          nrows = kRatio;
+          if (j < 0 || j >= s.nb) {
+            flag(a.st, QSA_DEV_BAD_SEL);
+            ok = false;
+          }
+        } else {
+          j = s.nb;
+          nrows = s.t;
+        }
+        if (ok) {
+          const int phys = a.bt[(int64_t)s.seq * a.mpps + j / kBlocksPerPage];
+          if (phys < 0 || phys >= a.num_pages) {
+            flag(a.st, QSA_DEV_BAD_PAGE);
+            ok = false;
+          } else {
+            off = (((size_t)phys * a.hkv + s.g) * kPage + (size_t)(j % kBlocksPerPage) * kRatio) * kHeadDim;
+          }
+        }
+        copy = ok;
+        rows = ok ? ((1u << nrows) - 1u) : 0u;
+      }
+      const int tiles = min(8, (s.n_valid - ub + kUnitsPerTile - 1) / kUnitsPerTile);
+      for (int tb = 0; tb < tiles; ++tb, ++T) {
+        const int stage = (int)(T % kStages);
+        if (T >= kStages) {
+          bool ok = true;
+          if (lane == 0) ok = mbar_wait_bounded(bar_empty + stage * 8, (uint32_t)((T / kStages - 1) & 1), kWaitLimitNs);
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok || *abort_flag) {
+            if (lane == 0 && !ok) {
+              flag(a.st, QSA_DEV_TIMEOUT);
+              *abort_flag = 1;
+            }
+            aborted = true;
+            break;
+          }
+        }
+        const bool mine = (lane >> 2) == tb;
+        const int slot = lane & 3;
+        const uint32_t bits = mine ? (rows << (slot * 4)) : 0u;
+        const bool do_copy = mine && copy;
+        const uint32_t rowmask = __reduce_or_sync(0xffffffffu, bits);
+        const uint32_t ncopy = __popc(__ballot_sync(0xffffffffu, do_copy));
+        if (lane == 0) {
+          meta[stage] = rowmask;
+          mbar_arrive_expect_tx(bar_full + stage * 8, ncopy * 2u * kUnitBytes);
+        }
+        __syncwarp();
+        if (do_copy) {
+          const uint32_t dk = ring + stage * kStageBytes + slot * kSlotStride;
+          bulk_g2s(dk, a.k_pages + off, kUnitBytes, bar_full + stage * 8, policy);
+          bulk_g2s(dk + kUnitsPerTile * kSlotStride, a.v_pages + off, kUnitBytes, bar_full + stage * 8, policy);
+        }
+      }
+    }
+  }
+  // Never leave the CTA with copies in flight: wait for the last tiles' data.
+  if (lane == 0) {
+    for (int64_t k = T > kStages ? T - kStages : 0; k < T; ++k)
+      mbar_wait_bounded(bar_full + (int)(k % kStages) * 8, (uint32_t)((k / kStages) & 1), kWaitLimitNs);
+  }
+  __syncwarp();
+}
+
+// ------------------------------------------------------------------ consumers
+
+__device__ __forceinline__ bool consumer_wait(const DecodeArgs& a, uint32_t bar, uint32_t parity,
+                                              volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 255u) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        flag(a.st, QSA_DEV_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+__device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_t x1) {
+  const int tid = threadIdx.x;  // 0..127
+  const int warp = tid >> 5, lane = tid & 31;
+  const int gq = lane >> 2, tq = lane & 3;
+  const uint32_t ring = smem_u32(smem + kOffRing);
+  const uint32_t bar_full = smem_u32(smem + kOffBar);
+  const uint32_t bar_empty = bar_full + kStages * 8;
+  const uint32_t* meta = reinterpret_cast<const uint32_t*>(smem + kOffMeta);
+  float* comb = reinterpret_cast<float*>(smem + kOffComb);
+  float* ml = reinterpret_cast<float*>(smem + kOffML);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
+  const int64_t n_slots = (int64_t)a.K + 1;
+  const int G = a.G;
+
+  // K tile: S column n = gq of n-tile j is token (slot ks, row 2j + ke)
+  const int ke = gq & 1;
+  const int ks = ((gq >> 1) + 2 * ke) & 3;
+  const uint32_t k_off = ks * kSlotStride + ke * 512 + tq * 16;
+  // S/P columns held by this lane: n = 2tq + e -> (slot (tq + 2e) & 3, row 2j + e)
+  const int ps0 = tq, ps1 = (tq + 2) & 3;
+  // V tokens of the PV B fragment: (ps0,row0) (ps1,row1) (ps0,row2) (ps1,row3)
+  const uint32_t v_off0 = kUnitsPerTile * kSlotStride + ps0 * kSlotStride + 0 * 512 + gq * 16;
+  const uint32_t v_off1 = kUnitsPerTile * kSlotStride + ps1 * kSlotStride + 1 * 512 + gq * 16;
+  const uint32_t v_off2 = kUnitsPerTile * kSlotStride + ps0 * kSlotStride + 2 * 512 + gq * 16;
+  const uint32_t v_off3 = kUnitsPerTile * kSlotStride + ps1 * kSlotStride + 3 * 512 + gq * 16;
+  const int vb0 = ps0 * 4 + 0, vb1 = ps1 * 4 + 1, vb2 = ps0 * 4 + 2, vb3 = ps1 * 4 + 3;
+
+  int64_t T_base = 0;
+  int seg_idx = 0;
+  for (int64_t pair = x0 / n_slots; pair <= (x1 - 1) / n_slots; ++pair, ++seg_idx) {
+    const Seg s = make_seg(a, pair, x0, x1, tid == 0);
+    uint8_t* qbuf = smem + kOffQ + (seg_idx & 1) * kQBufBytes;
+    const uint32_t qb = smem_u32(qbuf);
+    // ---- stage Q rows of this KV group (rows >= G are zero)
+    for (int idx = tid; idx < 16 * 32; idx += kConsumerThreads) {
+      const int row = idx >> 5, c = idx & 31;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (row < G && s.query_ok)
+        v = ldg_nc(a.q + ((size_t)s.q * a.hq + (size_t)s.g * G + row) * kHeadDim + c * 8);
+      sts128(qb + row * kQRowStride + c * 16, v);
+    }
+    named_bar_sync(kBarConsumers, kConsumerThreads);
+
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    float o[32][4];
+#pragma unroll
+    for (int nt = 0; nt < 32; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+
+    for (int ti = warp; ti < s.n_tiles; ti += kConsumerWarps) {
+      const int64_t T = T_base + ti;
+      const int stage = (int)(T % kStages);
+      if (!*abort_flag) consumer_wait(a, bar_full + stage * 8, (uint32_t)((T / kStages) & 1), abort_flag);
+      const uint32_t mask = meta[stage];
+      const uint32_t kb = ring + stage * kStageBytes;
+
+      // ---- S = Q K^T : two n-tiles of 8 tokens, k = 256 dims in 16 steps
+      float sa[2][4], sb[2][4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) sa[j][c] = sb[j][c] = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint4 qa = lds128(qb + gq * kQRowStride + (4 * i + tq) * 16);
+        const uint4 qc = lds128(qb + (gq + 8) * kQRowStride + (4 * i + tq) * 16);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const uint4 kk = lds128(kb + k_off + j * 1024 + i * 64);
+          float(&acc)[4] = (i & 1) ? sb[j] : sa[j];
+          mma_bf16_16816(acc, qa.x, qc.x, qa.y, qc.y, kk.x, kk.y);
+          mma_bf16_16816(acc, qa.z, qc.z, qa.w, qc.w, kk.z, kk.w);
+        }
+      }
+      // ---- mask, online softmax (base-2 logits)
+      float z[2][4];
+      float r0 = -INFINITY, r1 = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const bool v0 = (mask >> (ps0 * 4 + 2 * j)) & 1u;      // column 2tq   -> (ps0, row 2j)
+        const bool v1 = (mask >> (ps1 * 4 + 2 * j + 1)) & 1u;  // column 2tq+1 -> (ps1, row 2j+1)
+        z[j][0] = v0 ? (sa[j][0] + sb[j][0]) * a.scale_log2 : -INFINITY;
+        z[j][1] = v1 ? (sa[j][1] + sb[j][1]) * a.scale_log2 : -INFINITY;
+        z[j][2] = v0 ? (sa[j][2] + sb[j][2]) * a.scale_log2 : -INFINITY;
+        z[j][3] = v1 ? (sa[j][3] + sb[j][3]) * a.scale_log2 : -INFINITY;
+        r0 = fmaxf(r0, fmaxf(z[j][0], z[j][1]));
+        r1 = fmaxf(r1, fmaxf(z[j][2], z[j][3]));
+      }
+      r0 = fmaxf(r0, __shfl_xor_sync(0xffffffffu, r0, 1));
+      r1 = fmaxf(r1, __shfl_xor_sync(0xffffffffu, r1, 1));
+      r0 = fmaxf(r0, __shfl_xor_sync(0xffffffffu, r0, 2));
+      r1 = fmaxf(r1, __shfl_xor_sync(0xffffffffu, r1, 2));
+      const float mn0 = fmaxf(m0, r0), mn1 = fmaxf(m1, r1);
+      // a tile whose units were all rejected as bad data keeps every logit at -inf
+      const float sub0 = mn0 == -INFINITY ? 0.f : mn0, sub1 = mn1 == -INFINITY ? 0.f : mn1;
+      const float al0 = exp2f(m0 - sub0), al1 = exp2f(m1 - sub1);
+      m0 = mn0;
+      m1 = mn1;
+      float pr[2][4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        pr[j][0] = exp2f(z[j][0] - sub0);
+        pr[j][1] = exp2f(z[j][1] - sub0);
+        pr[j][2] = exp2f(z[j][2] - sub1);
+        pr[j][3] = exp2f(z[j][3] - sub1);
+      }
+      l0 = l0 * al0 + ((pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]));
+      l1 = l1 * al1 + ((pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]));
+      if (al0 != 1.f || al1 != 1.f) {
+#pragma unroll
+        for (int nt = 0; nt < 32; ++nt) {
+          o[nt][0] *= al0;
+          o[nt][1] *= al0;
+          o[nt][2] *= al1;
+          o[nt][3] *= al1;
+        }
+      }
+      const uint32_t pa0 = pack_bf16(pr[0][0], pr[0][1]);
+      const uint32_t pa1 = pack_bf16(pr[0][2], pr[0][3]);
+      const uint32_t pa2 = pack_bf16(pr[1][0], pr[1][1]);
+      const uint32_t pa3 = pack_bf16(pr[1][2], pr[1][3]);
+
+      // ---- O += P V : 32 n-tiles over the 256 output dims, k = the tile's 16 tokens
+      const bool full = mask == 0xffffu;
+      const bool ok0 = (mask >> vb0) & 1u, ok1 = (mask >> vb1) & 1u;
+      const bool ok2 = (mask >> vb2) & 1u, ok3 = (mask >> vb3) & 1u;
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) {
+        uint4 x0v = lds128(kb + v_off0 + qq * 128);
+        uint4 x1v = lds128(kb + v_off1 + qq * 128);
+        uint4 x2v = lds128(kb + v_off2 + qq * 128);
+        uint4 x3v = lds128(kb + v_off3 + qq * 128);
+        if (!full) {  // masked rows may hold stale or never-written data
+          if (!ok0) x0v = make_uint4(0, 0, 0, 0);
+          if (!ok1) x1v = make_uint4(0, 0, 0, 0);
+          if (!ok2) x2v = make_uint4(0, 0, 0, 0);
+          if (!ok3) x3v = make_uint4(0, 0, 0, 0);
+        }
+        const uint32_t a0[4] = {x0v.x, x0v.y, x0v.z, x0v.w};
+        const uint32_t a1[4] = {x1v.x, x1v.y, x1v.z, x1v.w};
+        const uint32_t a2[4] = {x2v.x, x2v.y, x2v.z, x2v.w};
+        const uint32_t a3[4] = {x3v.x, x3v.y, x3v.z, x3v.w};
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const uint32_t lo01 = __byte_perm(a0[r], a1[r], 0x5410);
+          const uint32_t hi01 = __byte_perm(a0[r], a1[r], 0x7632);
+          const uint32_t lo23 = __byte_perm(a2[r], a3[r], 0x5410);
+          const uint32_t hi23 = __byte_perm(a2[r], a3[r], 0x7632);
+          mma_bf16_16816(o[qq * 8 + 2 * r], pa0, pa1, pa2, pa3, lo01, lo23);
+          mma_bf16_16816(o[qq * 8 + 2 * r + 1], pa0, pa1, pa2, pa3, hi01, hi23);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_empty + stage * 8);
+    }
+    T_base += s.n_tiles;
+
+    // ---- merge the 4 warps' (m, l, O) and write the split partial
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    if (tq == 0) {
+      ml[(warp * 16 + gq) * 2 + 0] = m0;
+      ml[(warp * 16 + gq) * 2 + 1] = l0;
+      ml[(warp * 16 + gq + 8) * 2 + 0] = m1;
+      ml[(warp * 16 + gq + 8) * 2 + 1] = l1;
+    }
+    named_bar_sync(kBarConsumers, kConsumerThreads);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int row = gq + 8 * half;
+      if (row >= G) continue;
+      const float mine = half ? m1 : m0;
+      float M = -INFINITY;
+      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ml[(w * 16 + row) * 2]);
+      float fac = 0.f;
+      if (M != -INFINITY) {
+        float L = 0.f;
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float mw = ml[(w * 16 + row) * 2];
+          if (mw != -INFINITY) L += ml[(w * 16 + row) * 2 + 1] * exp2f(mw - M);
+        }
+        fac = mine != -INFINITY ? exp2f(mine - M) / L : 0.f;
+      }
+      float* dst = comb + (warp * 16 + row) * kCombRow;
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) {
+        // n-tile nt = 8qq + w8 holds dims 64qq + 16tq + w8 (c0/c2) and +8 (c1/c3)
+        float4* d4 = reinterpret_cast<float4*>(dst + 64 * qq + 16 * tq);
+        const int c_lo = half ? 2 : 0;
+        d4[0] = make_float4(o[qq * 8 + 0][c_lo] * fac, o[qq * 8 + 1][c_lo] * fac, o[qq * 8 + 2][c_lo] * fac,
+                            o[qq * 8 + 3][c_lo] * fac);
+        d4[1] = make_float4(o[qq * 8 + 4][c_lo] * fac, o[qq * 8 + 5][c_lo] * fac, o[qq * 8 + 6][c_lo] * fac,
+                            o[qq * 8 + 7][c_lo] * fac);
+        d4[2] = make_float4(o[qq * 8 + 0][c_lo + 1] * fac, o[qq * 8 + 1][c_lo + 1] * fac,
+                            o[qq * 8 + 2][c_lo + 1] * fac, o[qq * 8 + 3][c_lo + 1] * fac);
+        d4[3] = make_float4(o[qq * 8 + 4][c_lo + 1] * fac, o[qq * 8 + 5][c_lo + 1] * fac,
+                            o[qq * 8 + 6][c_lo + 1] * fac, o[qq * 8 + 7][c_lo + 1] * fac);
+      }
+    }
+    named_bar_sync(kBarConsumers, kConsumerThreads);
+    const size_t row0 = ((size_t)s.q * a.max_splits + s.split) * a.hq + (size_t)s.g * G;
+    for (int idx = tid; idx < G * 64; idx += kConsumerThreads) {
+      const int row = idx >> 6, c4 = idx & 63;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float4 v = *reinterpret_cast<const float4*>(comb + (w * 16 + row) * kCombRow + c4 * 4);
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      *reinterpret_cast<float4*>(a.part_o + (row0 + row) * kHeadDim + c4 * 4) = acc;
+    }
+    for (int row = tid; row < G; row += kConsumerThreads) {
+      float M = -INFINITY;
+      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ml[(w * 16 + row) * 2]);
+      float lse = -INFINITY;
+      if (M != -INFINITY) {
+        float L = 0.f;
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float mw = ml[(w * 16 + row) * 2];
+          if (mw != -INFINITY) L += ml[(w * 16 + row) * 2 + 1] * exp2f(mw - M);
+        }
+        lse = (M + log2f(L)) * 0.69314718055994530942f;
+      }
+      a.part_lse[row0 + row] = lse;
+    }
+    if (s.last_of_pair) {  // slots this pair never reaches: empty splits
+      for (int sp = s.split + 1; sp < a.max_splits; ++sp) {
+        const size_t r0 = ((size_t)s.q * a.max_splits + sp) * a.hq + (size_t)s.g * G;
+        for (int idx = tid; idx < G * 64; idx += kConsumerThreads)
+          *reinterpret_cast<float4*>(a.part_o + (r0 + (idx >> 6)) * kHeadDim + (idx & 63) * 4) =
+              make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int row = tid; row < G; row += kConsumerThreads) a.part_lse[r0 + row] = -INFINITY;
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(DecodeArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int64_t x0 = (int64_t)blockIdx.x * a.chunk;
+  const int64_t x1 = min(x0 + a.chunk, a.total_slots);
+  if (threadIdx.x == 0) {
+    const uint32_t bf = smem_u32(smem + kOffBar);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(bf + i * 8, 1);                  // full: producer's arrive + tx bytes
+      mbar_init(bf + (kStages + i) * 8, 1);      // empty: one consumer warp
+    }
+    *reinterpret_cast<volatile int*>(smem + kOffAbort) = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (x0 >= x1) return;
+  if (threadIdx.x >= kConsumerThreads)
+    producer(a, smem, x0, x1);
+  else
+    consumers(a, smem, x0, x1);
+}
+
+}  // namespace
+
+int32_t qsa_splits_bound(int32_t k, int32_t chunk);
+
+extern "C" int qsa_sparse_decode(const qsa_cache_t* cache, const void* q, int32_t nq, int32_t hq,
+                                 const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel,
+                                 const int32_t* count, int32_t k, float scale, int32_t chunk_units,
+                                 int32_t max_splits, float* part_o, float* part_lse, int32_t* dev_status,
+                                 void* stream) {
+  if (!cache || nq < 0 || hq < 1 || k < 0 || k > QSA_MAX_TOPK || chunk_units < 1 || max_splits < 1)
+    return QSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !(scale < 3.0e38f)) return QSA_ERR_INVALID_ARG;
+  const qsa_cache_t& c = *cache;
+  if (c.num_kv_heads < 1 || hq % c.num_kv_heads != 0) return QSA_ERR_INVALID_ARG;
+  if (hq / c.num_kv_heads > QSA_MAX_GROUP) return QSA_ERR_UNSUPPORTED;
+  if (max_splits < qsa_splits_bound(k, chunk_units)) return QSA_ERR_INVALID_ARG;
+  if (nq == 0) return QSA_OK;
+  if (!c.k_pages || !c.v_pages || !c.block_table || !q || !q_seq || !q_pos || !count || !part_o || !part_lse ||
+      (k > 0 && !sel))
+    return QSA_ERR_INVALID_ARG;
+  if (c.num_pages < 1 || c.max_seqs < 1 || c.max_pages_per_seq < 1) return QSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(c.k_pages) | reinterpret_cast<uintptr_t>(c.v_pages) |
+       reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(part_o)) & 15u)
+    return QSA_ERR_INVALID_ARG;
+  DecodeArgs a;
+  a.k_pages = static_cast<const __nv_bfloat16*>(c.k_pages);
+  a.v_pages = static_cast<const __nv_bfloat16*>(c.v_pages);
+  a.bt = c.block_table;
+  a.num_pages = c.num_pages;
+  a.max_seqs = c.max_seqs;
+  a.mpps = c.max_pages_per_seq;
+  a.hkv = c.num_kv_heads;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.hq = hq;
+  a.G = hq / c.num_kv_heads;
+  a.q_seq = q_seq;
+  a.q_pos = q_pos;
+  a.sel = sel;
+  a.count = count;
+  a.K = k;
+  a.scale_log2 = scale * 1.44269504088896340736f;
+  a.chunk = chunk_units;
+  a.total_slots = (int64_t)nq * c.num_kv_heads * ((int64_t)k + 1);
+  a.max_splits = max_splits;
+  a.part_o = part_o;
+  a.part_lse = part_lse;
+  a.st = dev_status;
+  const int64_t grid = (a.total_slots + a.chunk - 1) / a.chunk;
+  if (grid > 0x7fffffff) return QSA_ERR_UNSUPPORTED;
+  cudaError_t e = cudaFuncSetAttribute(sparse_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QSA_ERR_CUDA;
+  }
+  sparse_decode_kernel<<<(unsigned)grid, kThreads, kSmemBytes, static_cast<cudaStream_t>(stream)>>>(a);
+  return qsa_host::launch_status();
+}

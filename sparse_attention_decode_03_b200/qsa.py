@@ -1,0 +1,277 @@
+"""Thin ctypes binding of libqsa (include/qsa.h).
+
+Argument marshalling only: every step of the QSA decode path runs in the CUDA
+kernels of libqsa.so.  PyTorch supplies device memory and the current stream.
+The functions keep the C names; they take torch tensors, check dtype / device /
+shape / contiguity, pass raw pointers, and raise :class:`QSAError` on a
+non-zero status.  There is no fallback: if libqsa.so is missing, importing this
+module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqsa.so")
+
+HEAD_DIM = 256
+IDX_HEADS = 8
+IDX_DIM = 128
+RATIO = 4
+PAGE_TOKENS = 64
+BLOCKS_PER_PAGE = 16
+MAX_TOPK = 2048
+MAX_GROUP = 16
+
+QSA_OK, QSA_ERR_INVALID_ARG, QSA_ERR_UNSUPPORTED, QSA_ERR_CUDA = 0, -1, -2, -3
+DEV_BITS = {1: "BAD_PAGE", 2: "BAD_SEQ", 4: "BAD_POS", 8: "BAD_SEL", 16: "BAD_COUNT", 32: "BAD_ORDER",
+            64: "TIMEOUT", 128: "SCORES_LD"}
+
+
+class QSAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+        self.status = status
+
+
+class qsa_cache_t(ctypes.Structure):
+    _fields_ = [("k_pages", ctypes.c_void_p), ("v_pages", ctypes.c_void_p), ("kc_pages", ctypes.c_void_p),
+                ("kc_partial", ctypes.c_void_p), ("block_table", ctypes.c_void_p), ("num_pages", ctypes.c_int32),
+                ("max_seqs", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libqsa.so not built at {LIB_PATH}; run `python -m sparse_attention_decode_03_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+    PC = ctypes.POINTER(qsa_cache_t)
+    sig = {
+        "qsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "qsa_abi_version": (ctypes.c_int, []),
+        "qsa_append_kv": (ctypes.c_int, [PC, P, P, P, P, P, I32, P, P]),
+        "qsa_index_scores": (ctypes.c_int, [PC, P, P, P, P, I32, P, I64, P, P]),
+        "qsa_topk_blocks": (ctypes.c_int, [P, I64, P, I32, I32, P, P, P, P]),
+        "qsa_decode_plan": (ctypes.c_int, [I32, I32, I32, I32, ctypes.POINTER(I32), ctypes.POINTER(I32)]),
+        "qsa_sparse_decode": (ctypes.c_int, [PC, P, I32, I32, P, P, P, P, I32, F, I32, I32, P, P, P, P]),
+        "qsa_combine": (ctypes.c_int, [P, P, I32, I32, I32, P, P, P]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+LIB = _load()
+ABI_VERSION = LIB.qsa_abi_version()
+
+
+def status_string(status: int) -> str:
+    return LIB.qsa_status_string(int(status)).decode()
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != QSA_OK:
+        raise QSAError(fn, rc)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _req(t: torch.Tensor, name: str, dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None:
+        if t.dim() != len(shape) or any(s is not None and a != s for a, s in zip(t.shape, shape)):
+            raise ValueError(f"{name}: expected shape {shape}, got {tuple(t.shape)}")
+    return t
+
+
+# ----------------------------------------------------------------------------
+# cache group
+
+
+class PagedCache:
+    """Device buffers of one cache group: main K/V pages and the compressed-indexer
+    side cache, paged by the same page ids, plus the per-sequence open-block sum."""
+
+    def __init__(self, num_pages: int, max_seqs: int, max_pages_per_seq: int, num_kv_heads: int,
+                 block_table: torch.Tensor | None = None, device="cuda"):
+        dev = torch.device(device)
+        self.num_pages, self.max_seqs, self.max_pages_per_seq, self.num_kv_heads = (
+            int(num_pages), int(max_seqs), int(max_pages_per_seq), int(num_kv_heads))
+        self.k_pages = torch.empty((num_pages, num_kv_heads, PAGE_TOKENS, HEAD_DIM), dtype=torch.bfloat16, device=dev)
+        self.v_pages = torch.empty_like(self.k_pages)
+        self.kc_pages = torch.empty((num_pages, BLOCKS_PER_PAGE, IDX_DIM), dtype=torch.bfloat16, device=dev)
+        self.kc_partial = torch.zeros((max_seqs, IDX_DIM), dtype=torch.float32, device=dev)
+        if block_table is None:
+            block_table = torch.full((max_seqs, max_pages_per_seq), -1, dtype=torch.int32)
+        self.block_table = block_table.to(device=dev, dtype=torch.int32).contiguous()
+        assert tuple(self.block_table.shape) == (max_seqs, max_pages_per_seq)
+        self._struct = None
+
+    def struct(self) -> qsa_cache_t:
+        if self._struct is None:
+            self._struct = qsa_cache_t(self.k_pages.data_ptr(), self.v_pages.data_ptr(), self.kc_pages.data_ptr(),
+                                       self.kc_partial.data_ptr(), self.block_table.data_ptr(), self.num_pages,
+                                       self.max_seqs, self.max_pages_per_seq, self.num_kv_heads)
+        return self._struct
+
+    @property
+    def capacity_tokens(self) -> int:
+        return self.max_pages_per_seq * PAGE_TOKENS
+
+
+# ----------------------------------------------------------------------------
+# the five calls
+
+
+def qsa_append_kv(cache: PagedCache, k_new, v_new, kidx_new, seq_id, pos, dev_status=None, stream=None):
+    n = int(seq_id.shape[0]) if isinstance(seq_id, torch.Tensor) else -1
+    hkv = cache.num_kv_heads
+    _req(k_new, "k_new", torch.bfloat16, (n, hkv, HEAD_DIM))
+    _req(v_new, "v_new", torch.bfloat16, (n, hkv, HEAD_DIM))
+    _req(kidx_new, "kidx_new", torch.bfloat16, (n, IDX_DIM))
+    _req(seq_id, "seq_id", torch.int32, (n,))
+    _req(pos, "pos", torch.int32, (n,))
+    if dev_status is not None:
+        _req(dev_status, "dev_status", torch.int32, (1,))
+    _check("qsa_append_kv", LIB.qsa_append_kv(ctypes.byref(cache.struct()), _ptr(k_new), _ptr(v_new), _ptr(kidx_new),
+                                              _ptr(seq_id), _ptr(pos), n, _ptr(dev_status), _stream(stream)))
+
+
+def qsa_index_scores(cache: PagedCache, q_idx, w, q_seq, q_pos, scores, dev_status=None, stream=None):
+    nq = int(q_seq.shape[0])
+    _req(q_idx, "q_idx", torch.bfloat16, (nq, IDX_HEADS, IDX_DIM))
+    _req(w, "w", torch.float32, (nq, IDX_HEADS))
+    _req(q_seq, "q_seq", torch.int32, (nq,))
+    _req(q_pos, "q_pos", torch.int32, (nq,))
+    _req(scores, "scores", torch.float32, (nq, None))
+    if dev_status is not None:
+        _req(dev_status, "dev_status", torch.int32, (1,))
+    _check("qsa_index_scores", LIB.qsa_index_scores(ctypes.byref(cache.struct()), _ptr(q_idx), _ptr(w), _ptr(q_seq),
+                                                    _ptr(q_pos), nq, _ptr(scores), int(scores.shape[1]),
+                                                    _ptr(dev_status), _stream(stream)))
+
+
+def qsa_topk_blocks(scores, q_pos, k: int, sel, count, dev_status=None, stream=None):
+    nq = int(q_pos.shape[0])
+    _req(scores, "scores", torch.float32, (nq, None))
+    _req(q_pos, "q_pos", torch.int32, (nq,))
+    _req(sel, "sel", torch.int32, (nq, k))
+    _req(count, "count", torch.int32, (nq,))
+    if dev_status is not None:
+        _req(dev_status, "dev_status", torch.int32, (1,))
+    _check("qsa_topk_blocks", LIB.qsa_topk_blocks(_ptr(scores), int(scores.shape[1]), _ptr(q_pos), nq, int(k),
+                                                  _ptr(sel), _ptr(count), _ptr(dev_status), _stream(stream)))
+
+
+def qsa_decode_plan(nq: int, hkv: int, k: int, target_ctas: int) -> tuple[int, int]:
+    c, s = ctypes.c_int32(), ctypes.c_int32()
+    _check("qsa_decode_plan", LIB.qsa_decode_plan(int(nq), int(hkv), int(k), int(target_ctas), ctypes.byref(c),
+                                                  ctypes.byref(s)))
+    return c.value, s.value
+
+
+def qsa_sparse_decode(cache: PagedCache, q, q_seq, q_pos, sel, count, k: int, scale: float, chunk_units: int,
+                      max_splits: int, part_o, part_lse, dev_status=None, stream=None):
+    nq = int(q_seq.shape[0])
+    hq = int(q.shape[1]) if q.dim() == 3 else -1
+    _req(q, "q", torch.bfloat16, (nq, hq, HEAD_DIM))
+    _req(q_seq, "q_seq", torch.int32, (nq,))
+    _req(q_pos, "q_pos", torch.int32, (nq,))
+    _req(sel, "sel", torch.int32, (nq, k))
+    _req(count, "count", torch.int32, (nq,))
+    _req(part_o, "part_o", torch.float32, (nq, max_splits, hq, HEAD_DIM))
+    _req(part_lse, "part_lse", torch.float32, (nq, max_splits, hq))
+    if dev_status is not None:
+        _req(dev_status, "dev_status", torch.int32, (1,))
+    _check("qsa_sparse_decode", LIB.qsa_sparse_decode(
+        ctypes.byref(cache.struct()), _ptr(q), nq, hq, _ptr(q_seq), _ptr(q_pos), _ptr(sel), _ptr(count), int(k),
+        float(scale), int(chunk_units), int(max_splits), _ptr(part_o), _ptr(part_lse), _ptr(dev_status),
+        _stream(stream)))
+
+
+def qsa_combine(part_o, part_lse, out, lse, stream=None):
+    nq, S, hq = (int(x) for x in part_lse.shape)
+    _req(part_o, "part_o", torch.float32, (nq, S, hq, HEAD_DIM))
+    _req(part_lse, "part_lse", torch.float32, (nq, S, hq))
+    _req(out, "out", torch.bfloat16, (nq, hq, HEAD_DIM))
+    _req(lse, "lse", torch.float32, (nq, hq))
+    _check("qsa_combine", LIB.qsa_combine(_ptr(part_o), _ptr(part_lse), nq, S, hq, _ptr(out), _ptr(lse),
+                                          _stream(stream)))
+
+
+# ----------------------------------------------------------------------------
+# a decode step: the four calls on preallocated buffers
+
+
+class Decoder:
+    """Holds the per-step buffers (scores, selection, split partials, outputs) for
+    up to `max_nq` queries and runs index_scores -> topk -> sparse_decode ->
+    combine on the current stream, with no host synchronisation."""
+
+    def __init__(self, cache: PagedCache, hq: int, max_nq: int, k: int = 512, scale: float = 1.0 / 16.0,
+                 target_ctas: int | None = None, chunk_units: int | None = None, scores_ld: int | None = None):
+        dev = cache.k_pages.device
+        self.cache, self.hq, self.k, self.scale, self.max_nq = cache, hq, k, scale, max_nq
+        if target_ctas is None:
+            target_ctas = torch.cuda.get_device_properties(dev).multi_processor_count
+        if chunk_units is None:
+            chunk_units, self.max_splits = qsa_decode_plan(max_nq, cache.num_kv_heads, k, target_ctas)
+        else:
+            self.max_splits = splits_bound(k, chunk_units)
+        self.chunk_units = chunk_units
+        self.scores_ld = scores_ld or cache.max_pages_per_seq * BLOCKS_PER_PAGE
+        self.scores = torch.empty((max_nq, self.scores_ld), dtype=torch.float32, device=dev)
+        self.sel = torch.empty((max_nq, k), dtype=torch.int32, device=dev)
+        self.count = torch.empty((max_nq,), dtype=torch.int32, device=dev)
+        self.part_o = torch.empty((max_nq, self.max_splits, hq, HEAD_DIM), dtype=torch.float32, device=dev)
+        self.part_lse = torch.empty((max_nq, self.max_splits, hq), dtype=torch.float32, device=dev)
+        self.out = torch.empty((max_nq, hq, HEAD_DIM), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((max_nq, hq), dtype=torch.float32, device=dev)
+        self.dev_status = torch.zeros((1,), dtype=torch.int32, device=dev)
+
+    def run(self, q, q_idx, w, q_seq, q_pos, stream=None):
+        nq = int(q_seq.shape[0])
+        assert nq <= self.max_nq
+        sc, se, cn = self.scores[:nq], self.sel[:nq], self.count[:nq]
+        po, pl = self.part_o[:nq], self.part_lse[:nq]
+        qsa_index_scores(self.cache, q_idx, w, q_seq, q_pos, sc, self.dev_status, stream)
+        qsa_topk_blocks(sc, q_pos, self.k, se, cn, self.dev_status, stream)
+        qsa_sparse_decode(self.cache, q, q_seq, q_pos, se, cn, self.k, self.scale, self.chunk_units,
+                          self.max_splits, po, pl, self.dev_status, stream)
+        qsa_combine(po, pl, self.out[:nq], self.lse[:nq], stream)
+        return self.out[:nq], self.lse[:nq]
+
+
+def splits_bound(k: int, chunk_units: int) -> int:
+    """Most KV chunks one (query, KV head) pair's k+1 unit slots can touch."""
+    return (k + 1 + chunk_units - 2) // chunk_units + 1
+
+
+def dev_status_names(v: int) -> list[str]:
+    return [n for b, n in DEV_BITS.items() if v & b]
+
+
+def pages_for(tokens: int) -> int:
+    return math.ceil(tokens / PAGE_TOKENS)

@@ -1,0 +1,76 @@
+"""The C ABI without a GPU: the library loads, exports every entry point the
+header declares, and rejects bad arguments on the host before enqueuing work."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    txt = open(os.path.join(ROOT, "include", "qsa.h")).read()
+    return re.findall(r"QSA_API\s+[\w\s\*]+?\b(qsa_\w+)\s*\(", txt)
+
+
+def test_header_declares_the_five_calls():
+    names = set(header_functions())
+    for n in ("qsa_append_kv", "qsa_index_scores", "qsa_topk_blocks", "qsa_sparse_decode", "qsa_combine"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    import sparse_attention_decode_03_b200 as qsa
+    lib = ctypes.CDLL(qsa.LIB_PATH)
+    for n in header_functions():
+        assert hasattr(lib, n), n
+    assert qsa.ABI_VERSION == 1
+    assert qsa.status_string(0) == "QSA_OK" and qsa.status_string(-3) == "QSA_ERR_CUDA"
+
+
+def test_decode_plan():
+    import sparse_attention_decode_03_b200 as qsa
+    c, s = qsa.qsa_decode_plan(32, 2, 512, 148)
+    assert c == -(-32 * 2 * 513 // 148) and s == qsa.splits_bound(512, c)
+    c, s = qsa.qsa_decode_plan(1, 2, 512, 148)
+    assert c == 16 and s == (513 + 14) // 16 + 1
+    with pytest.raises(qsa.QSAError):
+        qsa.qsa_decode_plan(1, 0, 512, 148)
+    with pytest.raises(qsa.QSAError):
+        qsa.qsa_decode_plan(1, 1, 4096, 148)
+
+
+def test_host_validation_returns_before_any_cuda_call():
+    import sparse_attention_decode_03_b200 as qsa
+    L = qsa.qsa.LIB
+    fake = ctypes.c_void_p(0x1000)
+    cache = qsa.qsa.qsa_cache_t(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 10, 2, 4, 2)
+    cp = ctypes.byref(cache)
+    # sparse decode: Hq not a multiple of Hkv; group too large; K too large; too few split slots
+    args = lambda hq, k, chunk, ms: (cp, fake, 1, hq, fake, fake, fake, fake, k, 0.0625, chunk, ms, fake, fake, None, None)
+    assert L.qsa_sparse_decode(*args(3, 16, 16, 4)) == -1
+    assert L.qsa_sparse_decode(*args(64, 16, 16, 4)) == -2
+    assert L.qsa_sparse_decode(*args(16, 4096, 16, 400)) == -1
+    assert L.qsa_sparse_decode(*args(16, 512, 16, 2)) == -1
+    assert L.qsa_sparse_decode(None, fake, 1, 16, fake, fake, fake, fake, 16, 0.0625, 16, 4, fake, fake, None, None) == -1
+    assert L.qsa_sparse_decode(cp, fake, 1, 16, fake, fake, fake, fake, 16, 0.0, 16, 4, fake, fake, None, None) == -1
+    # zero queries is a no-op
+    assert L.qsa_sparse_decode(cp, fake, 0, 16, fake, fake, fake, fake, 16, 0.0625, 16, 4, fake, fake, None, None) == 0
+    assert L.qsa_topk_blocks(fake, 100, fake, 1, 4096, fake, fake, None, None) == -1
+    assert L.qsa_topk_blocks(fake, 0, fake, 1, 16, fake, fake, None, None) == -1
+    assert L.qsa_append_kv(cp, fake, fake, fake, fake, fake, -1, None, None) == -1
+    assert L.qsa_append_kv(cp, fake, fake, fake, fake, fake, 0, None, None) == 0
+    assert L.qsa_append_kv(None, fake, fake, fake, fake, fake, 5, None, None) == -1
+    assert L.qsa_index_scores(cp, None, fake, fake, fake, 1, fake, 16, None, None) == -1
+    assert L.qsa_combine(fake, fake, 1, 100, 128, fake, fake, None) == -2
+    assert L.qsa_combine(fake, fake, 1, 0, 16, fake, fake, None) == -1
+
+
+def test_binding_rejects_host_tensors():
+    import torch
+
+    import sparse_attention_decode_03_b200 as qsa
+    with pytest.raises(ValueError):
+        qsa.qsa_combine(torch.zeros(1, 2, 4, 256), torch.zeros(1, 2, 4), torch.zeros(1, 4, 256, dtype=torch.bfloat16),
+                        torch.zeros(1, 4))

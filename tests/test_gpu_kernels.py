@@ -1,0 +1,360 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle on small
+cases that still span several tiles, chunks and pages, plus the edge cases the
+pages' operator tests list ([CANN] "Negen tests ..."): unordered physical
+slots, several selection widths, default and explicit scales, fully masked
+rows, selection width zero, causal tail remainders 0..3, two requests sharing
+a prefix's physical pages, cache reuse, and the five local head shapes at 1 and
+257 query rows."""
+import dataclasses
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import qsa_oracle as O
+from tests import oracle_ref as R
+from workloads import configs as C
+
+pytestmark = pytest.mark.gpu
+
+qsa = pytest.importorskip("sparse_attention_decode_03_b200")
+H = pytest.importorskip("workloads.harness")
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _need_cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+
+
+def _status():
+    return torch.zeros(1, dtype=torch.int32, device="cuda")
+
+
+def run_step(wl, cache=None, k=None, chunk=None, scale=None, target_ctas=None):
+    st = _status()
+    if cache is None:
+        cache = H.build_cache(wl, dev_status=st)
+    inp = H.step_inputs(wl)
+    qsa.qsa_append_kv(cache, inp["k_new"], inp["v_new"], inp["kidx_new"], inp["seq_id"], inp["pos"], st)
+    dec = qsa.Decoder(cache, wl.hq, wl.nq, k=wl.k_top if k is None else k, scale=wl.scale if scale is None else scale,
+                      chunk_units=chunk, target_ctas=target_ctas)
+    dec.dev_status = st
+    dec.run(inp["q"], inp["q_idx"], inp["w"], inp["q_seq"], inp["q_pos"])
+    torch.cuda.synchronize()
+    return cache, dec, int(st.item())
+
+
+def bits16(t):
+    return t.contiguous().view(torch.int16).cpu()
+
+
+# ---------------------------------------------------------------- append
+
+
+def _append_irregular(cache, wl, st):
+    """Append every sequence's positions in irregular chunks, several
+    sequences per call, with padding tokens (seq_id -1) between the runs."""
+    sizes = [1, 3, 2, 64, 5, 100, 7, 250, 4, 1, 33]
+    cursor = [0] * wl.batch
+    it = 0
+    while any(c < L for c, L in zip(cursor, wl.lengths)):
+        parts = []
+        for b, L in enumerate(wl.lengths):
+            if cursor[b] >= L:
+                continue
+            n = min(sizes[(it + b) % len(sizes)], L - cursor[b])
+            pos = torch.arange(cursor[b], cursor[b] + n, device="cuda")
+            parts.append((C.k_rows(wl, b, pos, "cuda"), C.v_rows(wl, b, pos, "cuda"), C.kidx_rows(wl, b, pos, "cuda"),
+                          torch.full((n,), b, dtype=torch.int32, device="cuda"), pos.to(torch.int32)))
+            cursor[b] += n
+            # a padding token: garbage data, must write nothing
+            parts.append((torch.full((1, wl.hkv, 256), 999.0, dtype=torch.bfloat16, device="cuda"),
+                          torch.full((1, wl.hkv, 256), 999.0, dtype=torch.bfloat16, device="cuda"),
+                          torch.full((1, 128), 999.0, dtype=torch.bfloat16, device="cuda"),
+                          torch.full((1,), -1, dtype=torch.int32, device="cuda"),
+                          torch.zeros((1,), dtype=torch.int32, device="cuda")))
+        cat = [torch.cat([p[i] for p in parts]) for i in range(5)]
+        qsa.qsa_append_kv(cache, *cat, st)
+        it += 1
+
+
+@pytest.mark.parametrize("name,lengths", [("quarter", [301, 64, 130, 7]), ("long", [197, 260])])
+def test_append_kv_bit_exact(name, lengths):
+    wl = C.shrink(C.get(name), lengths, page_perm=True)
+    cache = H.new_cache(wl)
+    cache.k_pages.fill_(777.0)
+    cache.v_pages.fill_(777.0)
+    cache.kc_pages.fill_(555.0)
+    st = _status()
+    _append_irregular(cache, wl, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    bt = cache.block_table.cpu()
+    for b, L in enumerate(wl.lengths):
+        pos = torch.arange(L)
+        pg, row = bt[b, pos // 64].long(), pos % 64
+        k_gpu = cache.k_pages.cpu()[pg, :, row]
+        v_gpu = cache.v_pages.cpu()[pg, :, row]
+        assert torch.equal(k_gpu.view(torch.int16), C.k_rows(wl, b, pos).view(torch.int16))
+        assert torch.equal(v_gpu.view(torch.int16), C.v_rows(wl, b, pos).view(torch.int16))
+        kid = C.kidx_rows(wl, b, pos).float().numpy()
+        kc_ref = O.compress_keys(kid)
+        nb = L // 4
+        j = torch.arange(nb)
+        kc_gpu = cache.kc_pages.cpu()[bt[b, j // 16].long(), j % 16].float().numpy()
+        assert np.array_equal(kc_gpu.view(np.uint32), kc_ref.view(np.uint32))
+        if L % 4:
+            part = cache.kc_partial[b].cpu().numpy()
+            assert np.array_equal(part.view(np.uint32), O.open_block_partial(kid).view(np.uint32))
+        # untouched slots keep their sentinel
+        last = int(bt[b, (L - 1) // 64])
+        if L % 64:
+            assert torch.all(cache.k_pages[last, :, L % 64:].float() == 777.0)
+        if nb % 16:
+            assert torch.all(cache.kc_pages[last, nb % 16:].float() == 555.0)
+
+
+def test_append_chunking_is_bitwise_invariant():
+    """kc and the open-block partial do not depend on how the tokens are split
+    into calls (all at once vs one token per call)."""
+    wl = C.shrink(C.get("tiny"), [203])
+    a = H.new_cache(wl)
+    H.append_range(a, wl, 0, 0, 203)
+    b = H.new_cache(wl)
+    for p in range(203):
+        H.append_range(b, wl, 0, p, p + 1)
+    torch.cuda.synchronize()
+    bt = a.block_table.cpu()
+    j = torch.arange(203 // 4)
+    pos = torch.arange(203)
+    assert torch.equal(bits16(a.kc_pages.cpu()[bt[0, j // 16].long(), j % 16]),
+                       bits16(b.kc_pages.cpu()[bt[0, j // 16].long(), j % 16]))
+    assert torch.equal(a.kc_partial[0].cpu().view(torch.int32), b.kc_partial[0].cpu().view(torch.int32))
+    assert torch.equal(bits16(a.k_pages.cpu()[bt[0, pos // 64].long(), :, pos % 64]),
+                       bits16(b.k_pages.cpu()[bt[0, pos // 64].long(), :, pos % 64]))
+
+
+# ---------------------------------------------------------------- indexer + top-k
+
+
+@pytest.mark.parametrize("name,lengths,k", [
+    ("quarter", [4000, 999, 66, 5], 64),
+    ("long", [3000, 2050], 512),
+    ("batched", [1500], 16),
+    ("quarter", [700, 3], 0),
+])
+def test_index_scores_and_topk_bit_exact(name, lengths, k):
+    wl = C.shrink(C.get(name), lengths, page_perm=True, k_top=k)
+    cache, dec, st = run_step(wl, k=k)
+    assert st == 0
+    sc = dec.scores.cpu().numpy()
+    sel = dec.sel.cpu().numpy()
+    cnt = dec.count.cpu().numpy()
+    for row in range(wl.nq):
+        d = R.query_inputs(wl, row)
+        nb, _ = O.visible(d["p"])
+        kc = O.compress_keys(R.kidx_seq(wl, d["seq"], d["p"] + 1))
+        s_ref = O.block_scores(d["q_idx"], d["w"], kc)
+        assert np.array_equal(sc[row, :nb], s_ref.astype(np.float32)), f"scores row {row}"
+        sel_ref = O.select_blocks(s_ref, k)
+        assert cnt[row] == len(sel_ref)
+        assert np.array_equal(sel[row, :cnt[row]], sel_ref), f"selection row {row}"
+        assert np.all(sel[row, cnt[row]:] == -1)
+
+
+def test_topk_all_ties_take_lowest_indices():
+    wl = C.shrink(C.get("quarter"), [2000], k_top=100)
+    cache = H.new_cache(wl)
+    pos = torch.arange(0, 2000, device="cuda")
+    k = C.k_rows(wl, 0, pos, "cuda")
+    ki = torch.ones((2000, 128), dtype=torch.bfloat16, device="cuda")  # every kc equal
+    qsa.qsa_append_kv(cache, k, k, ki, torch.zeros(2000, dtype=torch.int32, device="cuda"), pos.to(torch.int32))
+    qs = C.queries(wl, device="cuda")
+    qs["q_pos"].fill_(1999)
+    dec = qsa.Decoder(cache, wl.hq, 1, k=100)
+    dec.run(qs["q"], qs["q_idx"], qs["w"], qs["q_seq"], qs["q_pos"])
+    torch.cuda.synchronize()
+    assert dec.count.item() == 100
+    assert dec.sel[0].tolist() == list(range(100))
+
+
+# ---------------------------------------------------------------- attention
+
+
+def _check_decode(wl, dec, rows, k=None, scale=None, chunk=None, prefix_from=None, partials=True):
+    out = dec.out.float().cpu().numpy()
+    lse = dec.lse.cpu().numpy()
+    po = dec.part_o.cpu().numpy()
+    pl = dec.part_lse.cpu().numpy()
+    sel = dec.sel.cpu().numpy()
+    for row in rows:
+        r = R.expect_query(wl, row, k=k, scale=scale, chunk=dec.chunk_units if partials else None,
+                           prefix_from=prefix_from)
+        assert np.array_equal(sel[row, :len(r["sel"])], r["sel"]), f"selection row {row}"
+        R.assert_close(out[row], r["o"], f"out row {row}")
+        R.assert_close(lse[row], r["lse"], f"lse row {row}")
+        if partials:
+            R.assert_close(po[row], r["part_o"], f"part_o row {row}")
+            R.assert_close(pl[row], r["part_lse"], f"part_lse row {row}")
+
+
+def _head_cases():
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "head_shapes.json")))
+    return [(hq, hkv, n) for hq, hkv in g["head_pairs"] for n in g["query_rows"]]
+
+
+@pytest.mark.parametrize("hq,hkv,nrows", _head_cases())
+def test_decode_head_shapes(hq, hkv, nrows):
+    base = C.get("quarter")
+    if nrows == 1:
+        wl = C.shrink(base, [3001], name=f"h{hq}x{hkv}", k_top=64)
+    else:  # 257 query rows: an extend of 257 tokens, every tail remainder
+        wl = C.shrink(base, [1200], new_tokens=nrows, name=f"h{hq}x{hkv}-extend", k_top=64)
+    wl = dataclasses.replace(wl, hq=hq, hkv=hkv, page_perm=True)
+    cache, dec, st = run_step(wl, k=64)
+    assert st == 0
+    rows = range(wl.nq) if wl.nq <= 8 else [0, 1, 2, 3, 100, 255, 256]
+    _check_decode(wl, dec, rows, k=64)
+
+
+@pytest.mark.parametrize("chunk", [1, 3, 16, 77, 513, 100000])
+def test_decode_chunk_sizes(chunk):
+    wl = C.shrink(C.get("long"), [2600, 1303], k_top=96)
+    cache, dec, st = run_step(wl, k=96, chunk=chunk)
+    assert st == 0
+    _check_decode(wl, dec, range(wl.nq), k=96)
+
+
+@pytest.mark.parametrize("k", [1, 15, 16, 17, 65])
+@pytest.mark.parametrize("tail", [0, 1, 2, 3])
+def test_decode_widths_and_tails(k, tail):
+    L = 4 * 300 + tail  # context incl. the query's own token
+    wl = C.shrink(C.get("batched"), [L - 1], k_top=k, page_perm=True)
+    cache, dec, st = run_step(wl, k=k)
+    assert st == 0
+    assert int(dec.count[0]) == k
+    _check_decode(wl, dec, [0], k=k)
+
+
+def test_explicit_scale():
+    wl = C.shrink(C.get("tiny"), [1999], k_top=40)
+    cache, dec, st = run_step(wl, k=40, scale=0.0371)
+    _check_decode(wl, dec, [0], k=40, scale=0.0371)
+
+
+def test_zero_budget_and_fully_masked_rows():
+    # K = 0: attention over the tail only; with t = 0 the row is fully masked
+    for L, t in ((4 * 50 + 2, 2), (4 * 50, 0)):
+        wl = C.shrink(C.get("tiny"), [L - 1], k_top=0)
+        cache, dec, st = run_step(wl, k=0)
+        assert st == 0 and int(dec.count[0]) == 0
+        if t == 0:
+            assert torch.all(dec.out == 0)
+            assert torch.all(torch.isneginf(dec.lse))
+        _check_decode(wl, dec, [0], k=0)
+
+
+def test_short_context_equals_dense():
+    # nb < K: every visible block is selected -> dense causal attention
+    wl = C.shrink(C.get("long"), [57, 6], k_top=512)
+    cache, dec, st = run_step(wl)
+    assert st == 0
+    assert dec.count.tolist() == [58 // 4, 7 // 4]
+    _check_decode(wl, dec, range(2))
+
+
+def test_shared_prefix_pages_and_cache_reuse():
+    """Two requests map a shared prefix onto the same physical pages; then the
+    cache is reused by a second decode step after more tokens are appended."""
+    wl = C.shrink(C.get("quarter"), [640 + 300, 640 + 901], k_top=48, page_perm=False)
+    wl2 = dataclasses.replace(wl, lengths=tuple(L + 1 + 37 for L in wl.lengths))
+    P = 10  # shared pages = 640 tokens
+    n0 = (wl2.total_lengths[0] + 63) // 64
+    n1 = (wl2.total_lengths[1] + 63) // 64
+    pps = max(n0, n1)
+    bt = torch.full((2, pps), -1, dtype=torch.int32)
+    bt[0, :n0] = torch.arange(n0)
+    bt[1, :P] = torch.arange(P)
+    bt[1, P:n1] = torch.arange(n0, n0 + n1 - P)
+    cache = qsa.PagedCache(num_pages=n0 + n1 - P, max_seqs=2, max_pages_per_seq=pps, num_kv_heads=wl.hkv,
+                           block_table=bt)
+    H.append_range(cache, wl, 0, 0, wl.lengths[0])          # writes the prefix once
+    H.append_range(cache, wl, 1, P * 64, wl.lengths[1])     # seq 1 only its own suffix
+    _, dec, st = run_step(wl, cache=cache, k=48)
+    assert st == 0
+    _check_decode(wl, dec, [0], k=48)
+    _check_decode(wl, dec, [1], k=48, prefix_from=(0, P * 64))
+    first = dec.out.clone()
+    # reuse: append 37 more tokens to both sequences and decode again
+    for b in range(2):
+        H.append_range(cache, wl, b, wl.lengths[b] + 1, wl2.lengths[b])
+    _, dec2, st = run_step(wl2, cache=cache, k=48)
+    assert st == 0
+    _check_decode(wl2, dec2, [0], k=48)
+    _check_decode(wl2, dec2, [1], k=48, prefix_from=(0, P * 64))
+    assert not torch.equal(first, dec2.out)
+
+
+def test_outputs_are_deterministic():
+    wl = C.shrink(C.get("long"), [5000, 4097, 2222], k_top=256)
+    cache, dec, st = run_step(wl, k=256)
+    inp = C.queries(wl, device="cuda")
+    outs = []
+    for _ in range(3):
+        dec.run(inp["q"], inp["q_idx"], inp["w"], inp["q_seq"], inp["q_pos"])
+        torch.cuda.synchronize()
+        outs.append((dec.out.clone(), dec.lse.clone(), dec.sel.clone(), dec.part_o.clone()))
+    for o in outs[1:]:
+        for a, b in zip(outs[0], o):
+            assert torch.equal(a.view(torch.uint8) if a.dtype != torch.int32 else a,
+                               b.view(torch.uint8) if b.dtype != torch.int32 else b)
+
+
+def test_device_status_flags_bad_data_without_faulting():
+    wl = C.shrink(C.get("quarter"), [900], k_top=32)
+    cache, dec, st = run_step(wl, k=32)
+    assert st == 0
+    inp = C.queries(wl, device="cuda")
+    # a selection index beyond the visible blocks and a count beyond K
+    sel = dec.sel.clone()
+    sel[0, 3] = 10 ** 6
+    s2 = _status()
+    qsa.qsa_sparse_decode(cache, inp["q"], inp["q_seq"], inp["q_pos"], sel, dec.count, 32, 1 / 16,
+                          dec.chunk_units, dec.max_splits, dec.part_o, dec.part_lse, s2)
+    torch.cuda.synchronize()
+    assert int(s2.item()) & 8
+    bad_count = torch.full_like(dec.count, 10 ** 6)
+    s3 = _status()
+    qsa.qsa_sparse_decode(cache, inp["q"], inp["q_seq"], inp["q_pos"], dec.sel, bad_count, 32, 1 / 16,
+                          dec.chunk_units, dec.max_splits, dec.part_o, dec.part_lse, s3)
+    torch.cuda.synchronize()
+    assert int(s3.item()) & 16
+    # a block-table entry outside the page pool
+    cache.block_table[0, 2] = 10 ** 7
+    s4 = _status()
+    qsa.qsa_index_scores(cache, inp["q_idx"], inp["w"], inp["q_seq"], inp["q_pos"], dec.scores, s4)
+    qsa.qsa_topk_blocks(dec.scores, inp["q_pos"], 32, dec.sel, dec.count, s4)
+    qsa.qsa_sparse_decode(cache, inp["q"], inp["q_seq"], inp["q_pos"], dec.sel, dec.count, 32, 1 / 16,
+                          dec.chunk_units, dec.max_splits, dec.part_o, dec.part_lse, s4)
+    torch.cuda.synchronize()
+    assert int(s4.item()) & 1
+    # the context is still usable
+    cache.block_table[0, 2] = C.block_table(wl)[0, 2]
+    dec.run(inp["q"], inp["q_idx"], inp["w"], inp["q_seq"], inp["q_pos"])
+    torch.cuda.synchronize()
+    _check_decode(wl, dec, [0], k=32)
+
+
+def test_host_errors_enqueue_nothing():
+    wl = C.shrink(C.get("tiny"), [300], k_top=16)
+    cache, dec, st = run_step(wl, k=16)
+    inp = C.queries(wl, device="cuda")
+    with pytest.raises(qsa.QSAError) as e:
+        qsa.qsa_sparse_decode(cache, inp["q"], inp["q_seq"], inp["q_pos"], dec.sel, dec.count, 16, 1 / 16,
+                              dec.chunk_units, 1, dec.part_o[:, :1], dec.part_lse[:, :1])
+    assert e.value.status == -1
+    with pytest.raises(ValueError):
+        qsa.qsa_index_scores(cache, inp["q_idx"].cpu(), inp["w"], inp["q_seq"], inp["q_pos"], dec.scores)
