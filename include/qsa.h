@@ -194,8 +194,9 @@ QSA_API int qsa_decode_plan(int32_t nq, int32_t hkv, int32_t k, int32_t target_c
  * (k, chunk_units), scale > 0 (the pages keep the D256 scale 1/16).
  * The kernel gathers each selected micro-block (4 tokens x 512 B of K and of V
  * per KV head, contiguous in a page) with bulk async copies into shared memory
- * and runs QK^T and PV on the tensor cores with fp32 accumulation; P is
- * rounded to BF16 for PV.
+ * and runs QK^T and PV on the tensor cores with fp32 accumulation; the
+ * softmax weights P enter PV as a BF16 hi + lo pair (about 17 significant
+ * bits), so short token sets keep full accuracy.
  */
 QSA_API int qsa_sparse_decode(const qsa_cache_t* cache, const void* q, int32_t nq, int32_t hq, const int32_t* q_seq,
                       const int32_t* q_pos, const int32_t* sel, const int32_t* count, int32_t k, float scale,

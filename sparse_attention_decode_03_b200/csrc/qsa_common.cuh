@@ -70,6 +70,15 @@ QSA_DEVINL uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// (a, b) -> hi = BF16x2(a, b) and lo = BF16x2 of the rounding residuals, so that
+// hi + lo carries about 17 significant bits of each value.
+QSA_DEVINL void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16(a, b);
+  const float ah = __uint_as_float(hi << 16);
+  const float bh = __uint_as_float(hi & 0xffff0000u);
+  lo = pack_bf16(a - ah, b - bh);
+}
+
 // ---------------------------------------------------------------- mbarrier + bulk copy
 
 QSA_DEVINL void mbar_init(uint32_t bar, uint32_t count) {

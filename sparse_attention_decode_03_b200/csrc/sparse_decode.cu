@@ -347,10 +347,13 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
           o[nt][3] *= al1;
         }
       }
-      const uint32_t pa0 = pack_bf16(pr[0][0], pr[0][1]);
-      const uint32_t pa1 = pack_bf16(pr[0][2], pr[0][3]);
-      const uint32_t pa2 = pack_bf16(pr[1][0], pr[1][1]);
-      const uint32_t pa3 = pack_bf16(pr[1][2], pr[1][3]);
+      // P = hi + lo, both BF16: the PV product keeps ~17 significant bits of
+      // every weight (BF16 alone, 8 bits, is too coarse for short token sets)
+      uint32_t pa[4], pl[4];
+      split_bf16(pr[0][0], pr[0][1], pa[0], pl[0]);
+      split_bf16(pr[0][2], pr[0][3], pa[1], pl[1]);
+      split_bf16(pr[1][0], pr[1][1], pa[2], pl[2]);
+      split_bf16(pr[1][2], pr[1][3], pa[3], pl[3]);
 
       // ---- O += P V : 32 n-tiles over the 256 output dims, k = the tile's 16 tokens
       const bool full = mask == 0xffffu;
@@ -378,8 +381,10 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
           const uint32_t hi01 = __byte_perm(a0[r], a1[r], 0x7632);
           const uint32_t lo23 = __byte_perm(a2[r], a3[r], 0x5410);
           const uint32_t hi23 = __byte_perm(a2[r], a3[r], 0x7632);
-          mma_bf16_16816(o[qq * 8 + 2 * r], pa0, pa1, pa2, pa3, lo01, lo23);
-          mma_bf16_16816(o[qq * 8 + 2 * r + 1], pa0, pa1, pa2, pa3, hi01, hi23);
+          mma_bf16_16816(o[qq * 8 + 2 * r], pa[0], pa[1], pa[2], pa[3], lo01, lo23);
+          mma_bf16_16816(o[qq * 8 + 2 * r], pl[0], pl[1], pl[2], pl[3], lo01, lo23);
+          mma_bf16_16816(o[qq * 8 + 2 * r + 1], pa[0], pa[1], pa[2], pa[3], hi01, hi23);
+          mma_bf16_16816(o[qq * 8 + 2 * r + 1], pl[0], pl[1], pl[2], pl[3], hi01, hi23);
         }
       }
       __syncwarp();

@@ -85,9 +85,9 @@ def _append_irregular(cache, wl, st):
 def test_append_kv_bit_exact(name, lengths):
     wl = C.shrink(C.get(name), lengths, page_perm=True)
     cache = H.new_cache(wl)
-    cache.k_pages.fill_(777.0)
-    cache.v_pages.fill_(777.0)
-    cache.kc_pages.fill_(555.0)
+    cache.k_pages.fill_(1024.0)
+    cache.v_pages.fill_(1024.0)
+    cache.kc_pages.fill_(512.0)
     st = _status()
     _append_irregular(cache, wl, st)
     torch.cuda.synchronize()
@@ -112,9 +112,9 @@ def test_append_kv_bit_exact(name, lengths):
         # untouched slots keep their sentinel
         last = int(bt[b, (L - 1) // 64])
         if L % 64:
-            assert torch.all(cache.k_pages[last, :, L % 64:].float() == 777.0)
+            assert torch.all(cache.k_pages[last, :, L % 64:].float() == 1024.0)
         if nb % 16:
-            assert torch.all(cache.kc_pages[last, nb % 16:].float() == 555.0)
+            assert torch.all(cache.kc_pages[last, nb % 16:].float() == 512.0)
 
 
 def test_append_chunking_is_bitwise_invariant():
