@@ -43,10 +43,12 @@ FALLBACK_HBM_GBS = 6650.0
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default="long", choices=list(C.ALL))
+    ap.add_argument("--batch", type=int, default=0, help="use only the first N sequences (profiling a small case)")
+    ap.add_argument("--context", type=int, default=0, help="override every context length (profiling a small case)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time budget for the CPU baseline")
     return ap.parse_args()
@@ -97,55 +99,69 @@ def dist_close(ws):
 
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples the SM clock and the clock-event (throttle) reasons of one GPU
+    through NVML (the counters nvidia-smi prints) every ~2 ms in a background
+    thread while the timed region runs."""
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.samples = []
+        self.max_mhz = None
+        self.ok = False
+
+    def _handle(self, nv):
+        try:
+            pci = torch.cuda.get_device_properties(self.dev)
+            bus = f"{pci.pci_domain_id:08X}:{pci.pci_bus_id:02X}:{pci.pci_device_id:02X}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:  # noqa: BLE001
+            return nv.nvmlDeviceGetHandleByIndex(self.dev)
 
     def __enter__(self):
+        import threading
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-i", str(self.gpu), "-lms", "200"], stdout=self.fh,
-                                         stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nv = nv
+            self.h = self._handle(nv)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # noqa: BLE001
+            return self
+        self.stop = threading.Event()
+
+        def loop():
+            nv, h = self.nv, self.h
+            while not self.stop.is_set():
+                try:
+                    mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                    reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((mhz, reasons))
+                except Exception:  # noqa: BLE001
+                    pass
+                time.sleep(0.002)
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.fh.close()
+        if self.ok:
+            self.stop.set()
+            self.thread.join(timeout=5)
 
     def summary(self):
-        if self.proc is None or not os.path.exists(self.path):
+        if not self.ok or not self.samples:
             return None
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "samples": len(sm), "reasons": sorted(reasons)}
+        reasons = set()
+        for _, r in self.samples:
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples), "reasons": sorted(reasons), "source": "NVML, 2 ms period"}
 
 
 # ---------------------------------------------------------------- algorithmic bytes
@@ -273,6 +289,10 @@ def run_native(args, rank, ws, local):
     from workloads import harness as H
 
     wl = C.get(args.workload)
+    if args.batch:
+        wl = C.shrink(wl, list(wl.lengths[:args.batch]), name=f"{wl.name}-first{args.batch}")
+    if args.context:
+        wl = C.shrink(wl, [args.context - wl.new_tokens] * wl.batch, name=f"{wl.name}-ctx{args.context}")
     dev = torch.device("cuda", local)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     st = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -286,26 +306,16 @@ def run_native(args, rank, ws, local):
     stream = torch.cuda.current_stream()
     names = ["append_kv", "index_scores", "topk", "sparse_decode", "combine"]
 
+    calls = [qsa.bind_append_kv(cache, inp["k_new"], inp["v_new"], inp["kidx_new"], inp["seq_id"], inp["pos"], st)]
+    calls += dec.bind(inp["q"], inp["q_idx"], inp["w"], inp["q_seq"], inp["q_pos"])
+
     def step(evs=None):
+        for k, call in enumerate(calls):
+            if evs:
+                evs[k].record()
+            call()
         if evs:
-            evs[0].record()
-        qsa.qsa_append_kv(cache, inp["k_new"], inp["v_new"], inp["kidx_new"], inp["seq_id"], inp["pos"], st)
-        if evs:
-            evs[1].record()
-        nq = wl.nq
-        qsa.qsa_index_scores(cache, inp["q_idx"], inp["w"], inp["q_seq"], inp["q_pos"], dec.scores[:nq], st)
-        if evs:
-            evs[2].record()
-        qsa.qsa_topk_blocks(dec.scores[:nq], inp["q_pos"], wl.k_top, dec.sel[:nq], dec.count[:nq], st)
-        if evs:
-            evs[3].record()
-        qsa.qsa_sparse_decode(cache, inp["q"], inp["q_seq"], inp["q_pos"], dec.sel[:nq], dec.count[:nq], wl.k_top,
-                              wl.scale, dec.chunk_units, dec.max_splits, dec.part_o[:nq], dec.part_lse[:nq], st)
-        if evs:
-            evs[4].record()
-        qsa.qsa_combine(dec.part_o[:nq], dec.part_lse[:nq], dec.out[:nq], dec.lse[:nq])
-        if evs:
-            evs[5].record()
+            evs[len(calls)].record()
 
     def between():
         cache.kc_partial.copy_(saved_partial)
@@ -330,6 +340,9 @@ def run_native(args, rank, ws, local):
         torch.cuda.synchronize()
         wall = time.perf_counter() - wall0
     barrier(ws)
+    status = int(st.item())
+    if status:
+        raise RuntimeError(f"device status after the timed steps: {qsa.dev_status_names(status)}")
     step_ms = [evs[i][0].elapsed_time(evs[i][5]) for i in range(args.steps)]
     kern_ms = {n: statistics.mean(evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(args.steps))
                for k, n in enumerate(names)}
@@ -359,6 +372,9 @@ def run_native(args, rank, ws, local):
             e2e_ms.append(e0.elapsed_time(e1))
         between()
     torch.cuda.synchronize()
+    status = int(st.item())
+    if status:
+        raise RuntimeError(f"device status after the e2e steps: {qsa.dev_status_names(status)}")
     e2e_total = max_over_ranks(sum(e2e_ms), ws)
     e2e_value = ws * wl.nq * len(e2e_ms) / (e2e_total / 1000.0)
 

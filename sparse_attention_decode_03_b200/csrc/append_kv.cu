@@ -38,9 +38,13 @@ struct AppendArgs {
 // Number of this call's tokens directly before `tok` that belong to the same
 // sequence at consecutive positions (at most `limit`).
 __device__ __forceinline__ int run_before(const AppendArgs& a, int64_t tok, int seq, int p, int limit) {
-  int m = 0;
-  while (m < limit && tok - m - 1 >= 0 && a.seq_id[tok - m - 1] == seq && a.pos[tok - m - 1] == p - m - 1) ++m;
-  return m;
+  bool same[3];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {  // independent loads, then the prefix test
+    const int64_t t = tok - k - 1;
+    same[k] = k < limit && t >= 0 && a.seq_id[t] == seq && a.pos[t] == p - k - 1;
+  }
+  return same[0] ? (same[1] ? (same[2] ? 3 : 2) : 1) : 0;
 }
 
 // fp32 running sum (4 dims per lane) of tokens tok-m .. tok, starting from

@@ -135,6 +135,11 @@ QSA_DEVINL void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t
       : "memory");
 }
 
+// Fire-and-forget prefetch of [src, src+bytes) into L2 (16-byte aligned, multiple of 16).
+QSA_DEVINL void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 QSA_DEVINL uint64_t l2_policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));

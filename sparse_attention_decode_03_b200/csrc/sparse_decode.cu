@@ -16,15 +16,19 @@
 // same number of slots whatever the batch shape.  The part of a pair inside a
 // chunk is a "segment"; each segment yields one split partial.
 //
-// CTA = 1 producer warp + 4 consumer warps, 1 CTA per SM.
-//   producer: looks up 32 units at a time (selection -> page table), then per
-//     tile of 4 units issues cp.async.bulk copies of the K and V micro-blocks
-//     into a 6-stage shared-memory ring (mbarrier full/empty pairs).
-//   consumers: each warp takes whole tiles (16 tokens) of the segment and runs
+// CTA = 4 consumer warps + a copy warp + a lookup warp, 1 CTA per SM.
+//   lookup warp: walks the CTA's units 32 at a time (selection -> page table),
+//     writes their source offsets into a 3-batch descriptor queue and prefetches
+//     the K and V micro-blocks into L2 (cp.async.bulk.prefetch.L2), so the
+//     page-table latency and most of the HBM latency sit ahead of the copies.
+//   copy warp: per tile of 4 units issues cp.async.bulk copies of the K and V
+//     micro-blocks (2 KiB each) into an 8-stage shared-memory ring
+//     (mbarrier full/empty pairs).
+//   consumers: tile T (16 tokens) belongs to warp T % 4; each warp runs
 //     S = Q K^T and O += P V with mma.sync m16n8k16 (M = 16 Q-head rows of the
 //     KV group, fp32 accumulate), online softmax in registers; at the end of a
-//     segment the 4 warps merge their (m, l, O) through shared memory and write
-//     the partial.
+//     segment the 4 warps merge their (m, l, O) in two rounds through shared
+//     memory and write the partial.
 // Shared-memory layouts are skewed so that every 16-byte fragment read is
 // bank-conflict free (micro-block slots 2080 B apart, Q rows 576 B apart).
 #include "qsa_common.cuh"
@@ -34,27 +38,41 @@ namespace {
 using namespace qsa;
 
 constexpr int kConsumerWarps = 4;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kCopyWarp = kConsumerWarps;         // warp 4
+constexpr int kLookupWarp = kConsumerWarps + 1;   // warp 5
+constexpr int kThreads = (kConsumerWarps + 2) * 32;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
-constexpr int kStages = 6;
+// A stage is reused by tile T + kStages; with kStages a multiple of the consumer
+// warp count and tile T owned by warp T % 4, that tile's owner is the warp that
+// consumed tile T, so no mbarrier wait can ever skip a phase (a parity wait can
+// only name the current phase or the one before it).
+constexpr int kStages = 8;
 constexpr int kUnitsPerTile = 4;
+constexpr int kBatch = 32;                                             // units per lookup batch
+constexpr int kDescSlots = 3;                                          // lookup batches in flight
 constexpr int kUnitBytes = kRatio * kHeadDim * 2;                      // 2048
 constexpr int kSlotStride = kUnitBytes + 32;                           // 2080
 constexpr int kStageBytes = 2 * kUnitsPerTile * kSlotStride;           // K slots then V slots
 constexpr int kQRowStride = kHeadDim * 2 + 64;                         // 576
 constexpr int kQBufBytes = 16 * kQRowStride;
 constexpr int kCombRow = kHeadDim + 4;                                 // floats
-constexpr int kCombBytes = kConsumerWarps * 16 * kCombRow * 4;
+constexpr int kCombBytes = 2 * 16 * kCombRow * 4;                      // two warps' O
 constexpr int kOffRing = 0;
 constexpr int kOffQ = kOffRing + kStages * kStageBytes;
-constexpr int kOffComb = kOffQ + 2 * kQBufBytes;
+constexpr int kOffComb = kOffQ + kQBufBytes;
 constexpr int kOffML = kOffComb + kCombBytes;
-constexpr int kOffMeta = kOffML + kConsumerWarps * 16 * 2 * 4;
+constexpr int kOffDescOff = kOffML + kConsumerWarps * 16 * 2 * 4;
+constexpr int kOffDescRows = kOffDescOff + kDescSlots * kBatch * 8;
+constexpr int kOffMeta = kOffDescRows + kDescSlots * kBatch * 4;
 constexpr int kOffBar = (kOffMeta + kStages * 4 + 7) & ~7;
-constexpr int kOffAbort = kOffBar + 2 * kStages * 8;
+constexpr int kNumBars = 2 * kStages + 2 * kDescSlots;
+constexpr int kOffAbort = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffAbort + 16;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kStages % kConsumerWarps == 0, "tile ownership must repeat with the stage ring");
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr int kBarConsumers = 1;                  // named barrier id
+constexpr uint64_t kNoCopy = ~0ull;
 
 struct DecodeArgs {
   const __nv_bfloat16* k_pages;
@@ -121,88 +139,181 @@ __device__ __forceinline__ Seg make_seg(const DecodeArgs& a, int64_t pair, int64
   return s;
 }
 
-// ------------------------------------------------------------------ producer
+// ------------------------------------------------------------------ producers
 
-__device__ void producer(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_t x1) {
+// Walk the CTA's segments in 32-unit batches (identical in both producer warps).
+struct BatchIter {
+  int64_t pair, last_pair, x0, x1;
+  int ub;
+  Seg s;
+};
+
+__device__ __forceinline__ bool iter_begin(const DecodeArgs& a, BatchIter& it, int64_t x0, int64_t x1) {
+  const int64_t n_slots = (int64_t)a.K + 1;
+  it.x0 = x0;
+  it.x1 = x1;
+  it.pair = x0 / n_slots;
+  it.last_pair = (x1 - 1) / n_slots;
+  it.ub = 0;
+  it.s = make_seg(a, it.pair, x0, x1, false);
+  while (it.s.n_valid == 0) {
+    if (++it.pair > it.last_pair) return false;
+    it.s = make_seg(a, it.pair, x0, x1, false);
+  }
+  return true;
+}
+
+__device__ __forceinline__ bool iter_next(const DecodeArgs& a, BatchIter& it) {
+  it.ub += kBatch;
+  while (it.ub >= it.s.n_valid) {
+    if (++it.pair > it.last_pair) return false;
+    it.s = make_seg(a, it.pair, it.x0, it.x1, false);
+    it.ub = 0;
+  }
+  return true;
+}
+
+// bounded wait used by the producer warps: lane 0 polls, the warp agrees
+__device__ __forceinline__ bool warp_wait(const DecodeArgs& a, uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  const int lane = threadIdx.x & 31;
+  int ok = 1;
+  if (lane == 0) {
+    ok = 0;
+    if (mbar_try_wait(bar, parity)) {
+      ok = 1;
+    } else {
+      const uint64_t t0 = global_timer_ns();
+      for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) {
+          ok = 1;
+          break;
+        }
+        if ((it & 255u) == 255u) {
+          if (*abort_flag) break;
+          if (global_timer_ns() - t0 > kWaitLimitNs) {
+            flag(a.st, QSA_DEV_TIMEOUT);
+            *abort_flag = 1;
+            break;
+          }
+        }
+      }
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();  // orders every lane after lane 0's acquire
+  return ok != 0;
+}
+
+// warp-uniform read of the abort flag
+__device__ __forceinline__ bool warp_aborted(volatile int* abort_flag) {
+  int v = 0;
+  if ((threadIdx.x & 31) == 0) v = *abort_flag;
+  return __shfl_sync(0xffffffffu, v, 0) != 0;
+}
+
+__device__ void lookup_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_t x1) {
+  const int lane = threadIdx.x & 31;
+  uint64_t* d_off = reinterpret_cast<uint64_t*>(smem + kOffDescOff);
+  uint32_t* d_rows = reinterpret_cast<uint32_t*>(smem + kOffDescRows);
+  const uint32_t bar_dfull = smem_u32(smem + kOffBar) + 2 * kStages * 8;
+  const uint32_t bar_dempty = bar_dfull + kDescSlots * 8;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
+  BatchIter it;
+  bool have = iter_begin(a, it, x0, x1);
+  for (int b = 0; have; ++b, have = iter_next(a, it)) {
+    const int slot = b % kDescSlots;
+    if (b >= kDescSlots && !warp_wait(a, bar_dempty + slot * 8, (uint32_t)((b / kDescSlots - 1) & 1), abort_flag))
+      return;
+    if (warp_aborted(abort_flag)) return;
+    const Seg& s = it.s;
+    const int i = it.ub + lane;
+    uint32_t rows = 0;
+    uint64_t off = kNoCopy;
+    if (i < s.n_valid) {
+      int j, nrows;
+      bool ok = true;
+      if (i < s.n_main) {
+        j = a.sel[(size_t)s.q * a.K + s.u0 + i];
+        nrows = kRatio;
+        if (j < 0 || j >= s.nb) {
+          flag(a.st, QSA_DEV_BAD_SEL);
+          ok = false;
+        }
+      } else {
+        j = s.nb;
+        nrows = s.t;
+      }
+      if (ok) {
+        const int phys = a.bt[(int64_t)s.seq * a.mpps + j / kBlocksPerPage];
+        if (phys < 0 || phys >= a.num_pages) {
+          flag(a.st, QSA_DEV_BAD_PAGE);
+        } else {
+          off = (((uint64_t)phys * a.hkv + s.g) * kPage + (uint64_t)(j % kBlocksPerPage) * kRatio) * kHeadDim;
+          rows = (1u << nrows) - 1u;
+          prefetch_l2(a.k_pages + off, kUnitBytes);
+          prefetch_l2(a.v_pages + off, kUnitBytes);
+        }
+      }
+    }
+    d_off[slot * kBatch + lane] = off;
+    d_rows[slot * kBatch + lane] = rows;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_dfull + slot * 8);
+  }
+}
+
+__device__ void copy_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_t x1) {
   const int lane = threadIdx.x & 31;
   const uint32_t ring = smem_u32(smem + kOffRing);
   const uint32_t bar_full = smem_u32(smem + kOffBar);
   const uint32_t bar_empty = bar_full + kStages * 8;
+  const uint32_t bar_dfull = bar_full + 2 * kStages * 8;
+  const uint32_t bar_dempty = bar_dfull + kDescSlots * 8;
+  const uint64_t* d_off = reinterpret_cast<const uint64_t*>(smem + kOffDescOff);
+  const uint32_t* d_rows = reinterpret_cast<const uint32_t*>(smem + kOffDescRows);
   uint32_t* meta = reinterpret_cast<uint32_t*>(smem + kOffMeta);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
   const uint64_t policy = l2_policy_evict_first();
-  const int64_t n_slots = (int64_t)a.K + 1;
   int64_t T = 0;
-  bool aborted = false;
-
-  for (int64_t pair = x0 / n_slots; pair <= (x1 - 1) / n_slots && !aborted; ++pair) {
-    const Seg s = make_seg(a, pair, x0, x1, false);
-    for (int ub = 0; ub < s.n_valid && !aborted; ub += 32) {
-      // lane i describes unit ub + i of the segment
-      const int i = ub + lane;
-      uint32_t rows = 0;
-      size_t off = 0;
-      bool copy = false;
-      if (i < s.n_valid) {
-        int j, nrows;
-        bool ok = true;
-        if (i < s.n_main) {
-          j = a.sel[(size_t)s.q * a.K + s.u0 + i];
-          nrows = kRatio;
-          if (j < 0 || j >= s.nb) {
-            flag(a.st, QSA_DEV_BAD_SEL);
-            ok = false;
-          }
-        } else {
-          j = s.nb;
-          nrows = s.t;
-        }
-        if (ok) {
-          const int phys = a.bt[(int64_t)s.seq * a.mpps + j / kBlocksPerPage];
-          if (phys < 0 || phys >= a.num_pages) {
-            flag(a.st, QSA_DEV_BAD_PAGE);
-            ok = false;
-          } else {
-            off = (((size_t)phys * a.hkv + s.g) * kPage + (size_t)(j % kBlocksPerPage) * kRatio) * kHeadDim;
-          }
-        }
-        copy = ok;
-        rows = ok ? ((1u << nrows) - 1u) : 0u;
+  BatchIter it;
+  bool have = iter_begin(a, it, x0, x1);
+  for (int b = 0; have; ++b, have = iter_next(a, it)) {
+    const int slot = b % kDescSlots;
+    if (!warp_wait(a, bar_dfull + slot * 8, (uint32_t)((b / kDescSlots) & 1), abort_flag)) break;
+    const uint64_t off = d_off[slot * kBatch + lane];
+    const uint32_t rows = d_rows[slot * kBatch + lane];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_dempty + slot * 8);
+    const int n_units = min(kBatch, it.s.n_valid - it.ub);
+    const int tiles = (n_units + kUnitsPerTile - 1) / kUnitsPerTile;
+    bool stop = false;
+    for (int tb = 0; tb < tiles; ++tb, ++T) {
+      const int stage = (int)(T % kStages);
+      if (T >= kStages && !warp_wait(a, bar_empty + stage * 8, (uint32_t)((T / kStages - 1) & 1), abort_flag)) {
+        stop = true;
+        break;
       }
-      const int tiles = min(8, (s.n_valid - ub + kUnitsPerTile - 1) / kUnitsPerTile);
-      for (int tb = 0; tb < tiles; ++tb, ++T) {
-        const int stage = (int)(T % kStages);
-        if (T >= kStages) {
-          bool ok = true;
-          if (lane == 0) ok = mbar_wait_bounded(bar_empty + stage * 8, (uint32_t)((T / kStages - 1) & 1), kWaitLimitNs);
-          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-          if (!ok || *abort_flag) {
-            if (lane == 0 && !ok) {
-              flag(a.st, QSA_DEV_TIMEOUT);
-              *abort_flag = 1;
-            }
-            aborted = true;
-            break;
-          }
-        }
-        const bool mine = (lane >> 2) == tb;
-        const int slot = lane & 3;
-        const uint32_t bits = mine ? (rows << (slot * 4)) : 0u;
-        const bool do_copy = mine && copy;
-        const uint32_t rowmask = __reduce_or_sync(0xffffffffu, bits);
-        const uint32_t ncopy = __popc(__ballot_sync(0xffffffffu, do_copy));
-        if (lane == 0) {
-          meta[stage] = rowmask;
-          mbar_arrive_expect_tx(bar_full + stage * 8, ncopy * 2u * kUnitBytes);
-        }
-        __syncwarp();
-        if (do_copy) {
-          const uint32_t dk = ring + stage * kStageBytes + slot * kSlotStride;
-          bulk_g2s(dk, a.k_pages + off, kUnitBytes, bar_full + stage * 8, policy);
-          bulk_g2s(dk + kUnitsPerTile * kSlotStride, a.v_pages + off, kUnitBytes, bar_full + stage * 8, policy);
-        }
+      if (warp_aborted(abort_flag)) {
+        stop = true;
+        break;
+      }
+      const bool mine = (lane >> 2) == tb && lane < n_units;
+      const int slot4 = lane & 3;
+      const bool do_copy = mine && off != kNoCopy;
+      const uint32_t rowmask = __reduce_or_sync(0xffffffffu, mine ? (rows << (slot4 * 4)) : 0u);
+      const uint32_t ncopy = __popc(__ballot_sync(0xffffffffu, do_copy));
+      if (lane == 0) {
+        meta[stage] = rowmask;
+        mbar_arrive_expect_tx(bar_full + stage * 8, ncopy * 2u * kUnitBytes);
+      }
+      __syncwarp();
+      if (do_copy) {
+        const uint32_t dk = ring + stage * kStageBytes + slot4 * kSlotStride;
+        bulk_g2s(dk, a.k_pages + off, kUnitBytes, bar_full + stage * 8, policy);
+        bulk_g2s(dk + kUnitsPerTile * kSlotStride, a.v_pages + off, kUnitBytes, bar_full + stage * 8, policy);
       }
     }
+    if (stop) break;
   }
   // Never leave the CTA with copies in flight: wait for the last tiles' data.
   if (lane == 0) {
@@ -262,7 +373,7 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
   int seg_idx = 0;
   for (int64_t pair = x0 / n_slots; pair <= (x1 - 1) / n_slots; ++pair, ++seg_idx) {
     const Seg s = make_seg(a, pair, x0, x1, tid == 0);
-    uint8_t* qbuf = smem + kOffQ + (seg_idx & 1) * kQBufBytes;
+    uint8_t* qbuf = smem + kOffQ;  // the merge barriers of the last segment order reuse
     const uint32_t qb = smem_u32(qbuf);
     // ---- stage Q rows of this KV group (rows >= G are zero)
     for (int idx = tid; idx < 16 * 32; idx += kConsumerThreads) {
@@ -279,10 +390,13 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
 #pragma unroll
     for (int nt = 0; nt < 32; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
 
-    for (int ti = warp; ti < s.n_tiles; ti += kConsumerWarps) {
+    // tile T (counted over the whole chunk) belongs to warp T % 4
+    const int first_ti = (int)(((int64_t)warp - T_base % kConsumerWarps + kConsumerWarps) % kConsumerWarps);
+    for (int ti = first_ti; ti < s.n_tiles; ti += kConsumerWarps) {
       const int64_t T = T_base + ti;
       const int stage = (int)(T % kStages);
       if (!*abort_flag) consumer_wait(a, bar_full + stage * 8, (uint32_t)((T / kStages) & 1), abort_flag);
+      __syncwarp();  // reconverge before the warp-wide mma.sync
       const uint32_t mask = meta[stage];
       const uint32_t kb = ring + stage * kStageBytes;
 
@@ -404,66 +518,84 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
       ml[(warp * 16 + gq + 8) * 2 + 1] = l1;
     }
     named_bar_sync(kBarConsumers, kConsumerThreads);
+    // this warp's weight for rows gq / gq+8, and the merged lse of those rows
+    float fac[2], lse_row[2];
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       const int row = gq + 8 * half;
-      if (row >= G) continue;
       const float mine = half ? m1 : m0;
       float M = -INFINITY;
       for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ml[(w * 16 + row) * 2]);
-      float fac = 0.f;
+      fac[half] = 0.f;
+      lse_row[half] = -INFINITY;
       if (M != -INFINITY) {
         float L = 0.f;
         for (int w = 0; w < kConsumerWarps; ++w) {
           const float mw = ml[(w * 16 + row) * 2];
           if (mw != -INFINITY) L += ml[(w * 16 + row) * 2 + 1] * exp2f(mw - M);
         }
-        fac = mine != -INFINITY ? exp2f(mine - M) / L : 0.f;
-      }
-      float* dst = comb + (warp * 16 + row) * kCombRow;
-#pragma unroll
-      for (int qq = 0; qq < 4; ++qq) {
-        // n-tile nt = 8qq + w8 holds dims 64qq + 16tq + w8 (c0/c2) and +8 (c1/c3)
-        float4* d4 = reinterpret_cast<float4*>(dst + 64 * qq + 16 * tq);
-        const int c_lo = half ? 2 : 0;
-        d4[0] = make_float4(o[qq * 8 + 0][c_lo] * fac, o[qq * 8 + 1][c_lo] * fac, o[qq * 8 + 2][c_lo] * fac,
-                            o[qq * 8 + 3][c_lo] * fac);
-        d4[1] = make_float4(o[qq * 8 + 4][c_lo] * fac, o[qq * 8 + 5][c_lo] * fac, o[qq * 8 + 6][c_lo] * fac,
-                            o[qq * 8 + 7][c_lo] * fac);
-        d4[2] = make_float4(o[qq * 8 + 0][c_lo + 1] * fac, o[qq * 8 + 1][c_lo + 1] * fac,
-                            o[qq * 8 + 2][c_lo + 1] * fac, o[qq * 8 + 3][c_lo + 1] * fac);
-        d4[3] = make_float4(o[qq * 8 + 4][c_lo + 1] * fac, o[qq * 8 + 5][c_lo + 1] * fac,
-                            o[qq * 8 + 6][c_lo + 1] * fac, o[qq * 8 + 7][c_lo + 1] * fac);
+        fac[half] = mine != -INFINITY ? exp2f(mine - M) / L : 0.f;
+        lse_row[half] = (M + log2f(L)) * 0.69314718055994530942f;
       }
     }
+#pragma unroll
+    for (int nt = 0; nt < 32; ++nt) {
+      o[nt][0] *= fac[0];
+      o[nt][1] *= fac[0];
+      o[nt][2] *= fac[1];
+      o[nt][3] *= fac[1];
+    }
+    // n-tile 8qq + w8 holds dims 64qq + 16tq + w8 (c0/c2) and 64qq + 16tq + 8 + w8 (c1/c3)
+    auto store_rows = [&](float* base, int row_stride) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int row = gq + 8 * half;
+        if (row >= G) continue;
+        const int c = 2 * half;
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          float4* d4 = reinterpret_cast<float4*>(base + (size_t)row * row_stride + 64 * qq + 16 * tq);
+          d4[0] = make_float4(o[qq * 8 + 0][c], o[qq * 8 + 1][c], o[qq * 8 + 2][c], o[qq * 8 + 3][c]);
+          d4[1] = make_float4(o[qq * 8 + 4][c], o[qq * 8 + 5][c], o[qq * 8 + 6][c], o[qq * 8 + 7][c]);
+          d4[2] = make_float4(o[qq * 8 + 0][c + 1], o[qq * 8 + 1][c + 1], o[qq * 8 + 2][c + 1], o[qq * 8 + 3][c + 1]);
+          d4[3] = make_float4(o[qq * 8 + 4][c + 1], o[qq * 8 + 5][c + 1], o[qq * 8 + 6][c + 1], o[qq * 8 + 7][c + 1]);
+        }
+      }
+    };
+    auto add_rows = [&](const float* base) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int row = gq + 8 * half;
+        if (row >= G) continue;
+        const int c = 2 * half;
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          const float4* s4 = reinterpret_cast<const float4*>(base + row * kCombRow + 64 * qq + 16 * tq);
+          const float4 x0 = s4[0], x1 = s4[1], x2 = s4[2], x3 = s4[3];
+          o[qq * 8 + 0][c] += x0.x; o[qq * 8 + 1][c] += x0.y; o[qq * 8 + 2][c] += x0.z; o[qq * 8 + 3][c] += x0.w;
+          o[qq * 8 + 4][c] += x1.x; o[qq * 8 + 5][c] += x1.y; o[qq * 8 + 6][c] += x1.z; o[qq * 8 + 7][c] += x1.w;
+          o[qq * 8 + 0][c + 1] += x2.x; o[qq * 8 + 1][c + 1] += x2.y; o[qq * 8 + 2][c + 1] += x2.z;
+          o[qq * 8 + 3][c + 1] += x2.w;
+          o[qq * 8 + 4][c + 1] += x3.x; o[qq * 8 + 5][c + 1] += x3.y; o[qq * 8 + 6][c + 1] += x3.z;
+          o[qq * 8 + 7][c + 1] += x3.w;
+        }
+      }
+    };
+    // round 1: warps 2, 3 hand their O to warps 0, 1; round 2: warp 1 to warp 0
+    if (warp >= 2) store_rows(comb + (warp - 2) * 16 * kCombRow, kCombRow);
+    named_bar_sync(kBarConsumers, kConsumerThreads);
+    if (warp < 2) add_rows(comb + warp * 16 * kCombRow);
+    named_bar_sync(kBarConsumers, kConsumerThreads);
+    if (warp == 1) store_rows(comb, kCombRow);
     named_bar_sync(kBarConsumers, kConsumerThreads);
     const size_t row0 = ((size_t)s.q * a.max_splits + s.split) * a.hq + (size_t)s.g * G;
-    for (int idx = tid; idx < G * 64; idx += kConsumerThreads) {
-      const int row = idx >> 6, c4 = idx & 63;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const float4 v = *reinterpret_cast<const float4*>(comb + (w * 16 + row) * kCombRow + c4 * 4);
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
+    if (warp == 0) {
+      add_rows(comb);
+      store_rows(a.part_o + row0 * kHeadDim, kHeadDim);
+      if (tq == 0) {
+        if (gq < G) a.part_lse[row0 + gq] = lse_row[0];
+        if (gq + 8 < G) a.part_lse[row0 + gq + 8] = lse_row[1];
       }
-      *reinterpret_cast<float4*>(a.part_o + (row0 + row) * kHeadDim + c4 * 4) = acc;
-    }
-    for (int row = tid; row < G; row += kConsumerThreads) {
-      float M = -INFINITY;
-      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ml[(w * 16 + row) * 2]);
-      float lse = -INFINITY;
-      if (M != -INFINITY) {
-        float L = 0.f;
-        for (int w = 0; w < kConsumerWarps; ++w) {
-          const float mw = ml[(w * 16 + row) * 2];
-          if (mw != -INFINITY) L += ml[(w * 16 + row) * 2 + 1] * exp2f(mw - M);
-        }
-        lse = (M + log2f(L)) * 0.69314718055994530942f;
-      }
-      a.part_lse[row0 + row] = lse;
     }
     if (s.last_of_pair) {  // slots this pair never reaches: empty splits
       for (int sp = s.split + 1; sp < a.max_splits; ++sp) {
@@ -484,16 +616,23 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(DecodeArgs a
   if (threadIdx.x == 0) {
     const uint32_t bf = smem_u32(smem + kOffBar);
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(bf + i * 8, 1);                  // full: producer's arrive + tx bytes
+      mbar_init(bf + i * 8, 1);                  // full: copy warp's arrive + tx bytes
       mbar_init(bf + (kStages + i) * 8, 1);      // empty: one consumer warp
+    }
+    for (int i = 0; i < kDescSlots; ++i) {
+      mbar_init(bf + (2 * kStages + i) * 8, 1);               // descriptors written (lookup warp)
+      mbar_init(bf + (2 * kStages + kDescSlots + i) * 8, 1);  // descriptors taken (copy warp)
     }
     *reinterpret_cast<volatile int*>(smem + kOffAbort) = 0;
     fence_mbar_init();
   }
   __syncthreads();
   if (x0 >= x1) return;
-  if (threadIdx.x >= kConsumerThreads)
-    producer(a, smem, x0, x1);
+  const int warp = threadIdx.x >> 5;
+  if (warp == kCopyWarp)
+    copy_warp(a, smem, x0, x1);
+  else if (warp == kLookupWarp)
+    lookup_warp(a, smem, x0, x1);
   else
     consumers(a, smem, x0, x1);
 }

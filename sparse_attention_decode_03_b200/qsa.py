@@ -222,6 +222,42 @@ def qsa_combine(part_o, part_lse, out, lse, stream=None):
 
 
 # ----------------------------------------------------------------------------
+# pre-bound launches: validate once, then call the C entry point directly
+
+
+class BoundCall:
+    """A C entry point with its arguments marshalled once.  Calling it only
+    enqueues the kernels (a few microseconds of host time), so a step of
+    several launches keeps the GPU fed.  The tensors must stay alive and
+    unchanged in shape while the call is used."""
+
+    def __init__(self, name: str, args: tuple, keep: tuple):
+        self.name = name
+        self.fn = getattr(LIB, name)
+        self.args = args
+        self._keep = keep  # tensors / structs referenced by raw pointers
+
+    def __call__(self):
+        rc = self.fn(*self.args)
+        if rc != QSA_OK:
+            raise QSAError(self.name, rc)
+
+
+def bind_append_kv(cache: PagedCache, k_new, v_new, kidx_new, seq_id, pos, dev_status=None, stream=None):
+    n = int(seq_id.shape[0])
+    hkv = cache.num_kv_heads
+    _req(k_new, "k_new", torch.bfloat16, (n, hkv, HEAD_DIM))
+    _req(v_new, "v_new", torch.bfloat16, (n, hkv, HEAD_DIM))
+    _req(kidx_new, "kidx_new", torch.bfloat16, (n, IDX_DIM))
+    _req(seq_id, "seq_id", torch.int32, (n,))
+    _req(pos, "pos", torch.int32, (n,))
+    st = cache.struct()
+    return BoundCall("qsa_append_kv", (ctypes.byref(st), _ptr(k_new), _ptr(v_new), _ptr(kidx_new), _ptr(seq_id),
+                                       _ptr(pos), n, _ptr(dev_status), _stream(stream)),
+                     (cache, st, k_new, v_new, kidx_new, seq_id, pos, dev_status))
+
+
+# ----------------------------------------------------------------------------
 # a decode step: the four calls on preallocated buffers
 
 
@@ -250,6 +286,34 @@ class Decoder:
         self.out = torch.empty((max_nq, hq, HEAD_DIM), dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty((max_nq, hq), dtype=torch.float32, device=dev)
         self.dev_status = torch.zeros((1,), dtype=torch.int32, device=dev)
+
+    def bind(self, q, q_idx, w, q_seq, q_pos, stream=None) -> list:
+        """Validate the step inputs once and return the four pre-bound launches
+        (index_scores, topk, sparse_decode, combine) for them."""
+        nq = int(q_seq.shape[0])
+        assert nq <= self.max_nq
+        hq = self.hq
+        _req(q_idx, "q_idx", torch.bfloat16, (nq, IDX_HEADS, IDX_DIM))
+        _req(w, "w", torch.float32, (nq, IDX_HEADS))
+        _req(q_seq, "q_seq", torch.int32, (nq,))
+        _req(q_pos, "q_pos", torch.int32, (nq,))
+        _req(q, "q", torch.bfloat16, (nq, hq, HEAD_DIM))
+        sc, se, cn = self.scores[:nq], self.sel[:nq], self.count[:nq]
+        po, pl = self.part_o[:nq], self.part_lse[:nq]
+        out, lse = self.out[:nq], self.lse[:nq]
+        st = self.cache.struct()
+        ds, sp = _ptr(self.dev_status), _stream(stream)
+        keep = (self.cache, st, q, q_idx, w, q_seq, q_pos, self.dev_status)
+        return [
+            BoundCall("qsa_index_scores", (ctypes.byref(st), _ptr(q_idx), _ptr(w), _ptr(q_seq), _ptr(q_pos), nq,
+                                           _ptr(sc), int(sc.shape[1]), ds, sp), keep),
+            BoundCall("qsa_topk_blocks", (_ptr(sc), int(sc.shape[1]), _ptr(q_pos), nq, self.k, _ptr(se), _ptr(cn),
+                                          ds, sp), keep),
+            BoundCall("qsa_sparse_decode", (ctypes.byref(st), _ptr(q), nq, hq, _ptr(q_seq), _ptr(q_pos), _ptr(se),
+                                            _ptr(cn), self.k, float(self.scale), self.chunk_units, self.max_splits,
+                                            _ptr(po), _ptr(pl), ds, sp), keep),
+            BoundCall("qsa_combine", (_ptr(po), _ptr(pl), nq, self.max_splits, hq, _ptr(out), _ptr(lse), sp), keep),
+        ]
 
     def run(self, q, q_idx, w, q_seq, q_pos, stream=None):
         nq = int(q_seq.shape[0])

@@ -63,7 +63,7 @@ def test_host_validation_returns_before_any_cuda_call():
     assert L.qsa_append_kv(cp, fake, fake, fake, fake, fake, 0, None, None) == 0
     assert L.qsa_append_kv(None, fake, fake, fake, fake, fake, 5, None, None) == -1
     assert L.qsa_index_scores(cp, None, fake, fake, fake, 1, fake, 16, None, None) == -1
-    assert L.qsa_combine(fake, fake, 1, 100, 128, fake, fake, None) == -2
+    assert L.qsa_combine(ctypes.c_void_p(0x1004), fake, 1, 4, 16, fake, fake, None) == -1  # misaligned
     assert L.qsa_combine(fake, fake, 1, 0, 16, fake, fake, None) == -1
 
 

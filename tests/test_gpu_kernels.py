@@ -358,3 +358,25 @@ def test_host_errors_enqueue_nothing():
     assert e.value.status == -1
     with pytest.raises(ValueError):
         qsa.qsa_index_scores(cache, inp["q_idx"].cpu(), inp["w"], inp["q_seq"], inp["q_pos"], dec.scores)
+
+
+def test_split_pipeline_stress_no_expired_waits():
+    """Hundreds of decode launches with an L2 flush between them: the copy /
+    consumer pipeline never loses a phase (a wait that named a stale phase
+    would consume unarrived data and later expire with the TIMEOUT bit), and
+    every launch reproduces the first one bit for bit."""
+    wl = C.shrink(C.get("long"), [16383] * 16, k_top=512)
+    cache, dec, st = run_step(wl)
+    assert st == 0
+    inp = C.queries(wl, device="cuda")
+    calls = dec.bind(inp["q"], inp["q_idx"], inp["w"], inp["q_seq"], inp["q_pos"])
+    ref_o, ref_l = dec.out.clone(), dec.part_lse.clone()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for _ in range(300):
+        calls[2]()
+        calls[3]()
+        flush.zero_()
+    torch.cuda.synchronize()
+    assert int(dec.dev_status.item()) == 0, qsa.dev_status_names(int(dec.dev_status.item()))
+    assert torch.equal(dec.out.view(torch.int16), ref_o.view(torch.int16))
+    assert torch.equal(dec.part_lse, ref_l)
