@@ -86,17 +86,20 @@ typedef enum {
  * One cache group ([DCP]: the selector and the main KV cache are kept in one
  * cache group so they cannot drift apart).  The main K/V and the compressed
  * indexer side cache are paged by the SAME physical page ids.
- *   k_pages, v_pages  bf16 [num_pages][num_kv_heads][64][256]  post-RoPE K / V
- *   kc_pages          bf16 [num_pages][16][128]  kc of the 16 micro-blocks of a page
- *   kc_partial        fp32 [max_seqs][128]       running fp32 sum of each sequence's
- *                                                 open (incomplete) micro-block
- *   block_table       int32 [max_seqs][max_pages_per_seq]  logical page -> physical page
- * All buffers are caller-owned device memory; the library writes k/v/kc pages
+ *   kv_pages    bf16 [num_pages][num_kv_heads][16][2][4][256]  post-RoPE K and V:
+ *               per page and KV head, its 16 micro-blocks of 4 tokens, each
+ *               holding the 4 K rows then the 4 V rows, so one selected
+ *               micro-block of one KV head is a single contiguous 4 KiB run
+ *               (token t of a page: micro-block t / 4, row t % 4)
+ *   kc_pages    bf16 [num_pages][16][128]  kc of the 16 micro-blocks of a page
+ *   kc_partial  fp32 [max_seqs][128]       running fp32 sum of each sequence's
+ *                                           open (incomplete) micro-block
+ *   block_table int32 [max_seqs][max_pages_per_seq]  logical page -> physical page
+ * All buffers are caller-owned device memory; the library writes kv/kc pages
  * and kc_partial only in qsa_append_kv.
  */
 typedef struct {
-  void* k_pages;
-  void* v_pages;
+  void* kv_pages;
   void* kc_pages;
   float* kc_partial;
   const int32_t* block_table;
@@ -111,7 +114,7 @@ QSA_API const char* qsa_status_string(int status);
 
 /* ABI version of this header (bumped on any signature change). */
 QSA_API int qsa_abi_version(void);
-#define QSA_ABI_VERSION 1
+#define QSA_ABI_VERSION 2
 
 /*
  * qsa_append_kv -- write n new tokens into the cache group.
@@ -120,7 +123,7 @@ QSA_API int qsa_abi_version(void);
  * the QSA side caches: a token with seq_id < 0 is skipped entirely.
  *   k_new, v_new  bf16 [n][Hkv][256];  kidx_new  bf16 [n][128] (indexer keys)
  *   seq_id, pos   int32 [n]  sequence and absolute position of each token
- * Effect: K/V rows written at page block_table[seq][pos/64], row pos%64.  The
+ * Effect: K/V rows written at page block_table[seq][pos/64], token pos%64.  The
  * indexer keys of a micro-block are summed in fp32 in token order (continuing
  * kc_partial when the block began in an earlier call); when the token at
  * position 4j+3 arrives, kc_pages row j = BF16(sum) (round to nearest even).
@@ -192,8 +195,8 @@ QSA_API int qsa_decode_plan(int32_t nq, int32_t hkv, int32_t k, int32_t target_c
  * Requirements: hq % Hkv == 0, hq / Hkv <= 16, 0 <= k <= QSA_MAX_TOPK,
  * chunk_units >= 1, max_splits >= the value qsa_decode_plan reports for
  * (k, chunk_units), scale > 0 (the pages keep the D256 scale 1/16).
- * The kernel gathers each selected micro-block (4 tokens x 512 B of K and of V
- * per KV head, contiguous in a page) with bulk async copies into shared memory
+ * The kernel gathers each selected micro-block (4 K rows + 4 V rows of one KV
+ * head: one contiguous 4 KiB run) with one bulk async copy into shared memory
  * and runs QK^T and PV on the tensor cores with fp32 accumulation; the
  * softmax weights P enter PV as a BF16 hi + lo pair (about 17 significant
  * bits), so short token sets keep full accuracy.

@@ -88,13 +88,14 @@ __global__ void __launch_bounds__(kWarps * 32) append_scatter_kernel(AppendArgs 
   }
   const int slot = p % kPage;
   const int hkv = a.c.num_kv_heads;
-  __nv_bfloat16* kp = static_cast<__nv_bfloat16*>(a.c.k_pages);
-  __nv_bfloat16* vp = static_cast<__nv_bfloat16*>(a.c.v_pages);
+  __nv_bfloat16* kv = static_cast<__nv_bfloat16*>(a.c.kv_pages);
   for (int h = 0; h < hkv; ++h) {
-    const size_t dst = (((size_t)page * hkv + h) * kPage + slot) * kHeadDim + lane * 8;
+    // [page][h][micro-block][K rows | V rows][256]
+    const size_t blk = (((size_t)page * hkv + h) * kBlocksPerPage + slot / kRatio) * (2 * kRatio * kHeadDim);
+    const size_t dst = blk + (size_t)(slot % kRatio) * kHeadDim + lane * 8;
     const size_t src = ((size_t)tok * hkv + h) * kHeadDim + lane * 8;
-    *reinterpret_cast<uint4*>(kp + dst) = *reinterpret_cast<const uint4*>(a.k_new + src);
-    *reinterpret_cast<uint4*>(vp + dst) = *reinterpret_cast<const uint4*>(a.v_new + src);
+    *reinterpret_cast<uint4*>(kv + dst) = *reinterpret_cast<const uint4*>(a.k_new + src);
+    *reinterpret_cast<uint4*>(kv + dst + kRatio * kHeadDim) = *reinterpret_cast<const uint4*>(a.v_new + src);
   }
   if ((p & 3) == 3) {  // this token closes micro-block p / 4
     const int m = run_before(a, tok, seq, p, 3);
@@ -135,10 +136,10 @@ extern "C" int qsa_append_kv(const qsa_cache_t* cache, const void* k_new, const 
   if (!cache || n < 0) return QSA_ERR_INVALID_ARG;
   if (n == 0) return QSA_OK;
   const qsa_cache_t& c = *cache;
-  if (!c.k_pages || !c.v_pages || !c.kc_pages || !c.kc_partial || !c.block_table) return QSA_ERR_INVALID_ARG;
+  if (!c.kv_pages || !c.kc_pages || !c.kc_partial || !c.block_table) return QSA_ERR_INVALID_ARG;
   if (!k_new || !v_new || !kidx_new || !seq_id || !pos) return QSA_ERR_INVALID_ARG;
   if (c.num_pages < 1 || c.max_seqs < 1 || c.max_pages_per_seq < 1 || c.num_kv_heads < 1) return QSA_ERR_INVALID_ARG;
-  if (!aligned16(c.k_pages) || !aligned16(c.v_pages) || !aligned16(c.kc_partial) || !aligned16(k_new) ||
+  if (!aligned16(c.kv_pages) || !aligned16(c.kc_partial) || !aligned16(k_new) ||
       !aligned16(v_new) || (reinterpret_cast<uintptr_t>(c.kc_pages) & 7u) || (reinterpret_cast<uintptr_t>(kidx_new) & 7u))
     return QSA_ERR_INVALID_ARG;
   AppendArgs a{c,

@@ -10,27 +10,28 @@
 // fully masked rows) and "Negen tests ..." (causal tail remainders 0..3).
 //
 // Work decomposition.  Each (query, KV head) pair owns K+1 unit slots: the K
-// selection slots (one micro-block of 4 tokens each, 2 KiB of K and 2 KiB of V
-// per KV head, contiguous in a page) and the tail slot.  All slots, query
+// selection slots (one micro-block of 4 tokens each: its 4 K rows and 4 V rows
+// of one KV head form one contiguous 4 KiB run in the cache) and the tail slot.  All slots, query
 // major, are cut into fixed chunks; one CTA per chunk, so every SM gets the
 // same number of slots whatever the batch shape.  The part of a pair inside a
 // chunk is a "segment"; each segment yields one split partial.
 //
 // CTA = 4 consumer warps + a copy warp + a lookup warp, 1 CTA per SM.
-//   lookup warp: walks the CTA's units 32 at a time (selection -> page table),
-//     writes their source offsets into a 3-batch descriptor queue and prefetches
-//     the K and V micro-blocks into L2 (cp.async.bulk.prefetch.L2), so the
-//     page-table latency and most of the HBM latency sit ahead of the copies.
-//   copy warp: per tile of 4 units issues cp.async.bulk copies of the K and V
-//     micro-blocks (2 KiB each) into an 8-stage shared-memory ring
-//     (mbarrier full/empty pairs).
+//   lookup warp: walks the CTA's units 32 at a time (selection -> page table)
+//     and writes their source offsets into a 3-batch descriptor queue, so the
+//     dependent selection and page-table loads run ahead of the copies.
+//   copy warp: per tile of 4 units issues one cp.async.bulk copy of 4 KiB per
+//     unit into an 8-stage shared-memory ring (mbarrier full/empty pairs).
+//     The bulk-copy engine costs about a hundred cycles per operation on B200,
+//     whatever its size; 4 KiB operations keep it near HBM speed where 2 KiB
+//     ones cap an SM at about two thirds of its share.
 //   consumers: tile T (16 tokens) belongs to warp T % 4; each warp runs
 //     S = Q K^T and O += P V with mma.sync m16n8k16 (M = 16 Q-head rows of the
 //     KV group, fp32 accumulate), online softmax in registers; at the end of a
 //     segment the 4 warps merge their (m, l, O) in two rounds through shared
 //     memory and write the partial.
 // Shared-memory layouts are skewed so that every 16-byte fragment read is
-// bank-conflict free (micro-block slots 2080 B apart, Q rows 576 B apart).
+// bank-conflict free (micro-block slots 4128 B apart, Q rows 576 B apart).
 #include "qsa_common.cuh"
 
 namespace {
@@ -50,9 +51,10 @@ constexpr int kStages = 8;
 constexpr int kUnitsPerTile = 4;
 constexpr int kBatch = 32;                                             // units per lookup batch
 constexpr int kDescSlots = 3;                                          // lookup batches in flight
-constexpr int kUnitBytes = kRatio * kHeadDim * 2;                      // 2048
-constexpr int kSlotStride = kUnitBytes + 32;                           // 2080
-constexpr int kStageBytes = 2 * kUnitsPerTile * kSlotStride;           // K slots then V slots
+constexpr int kHalfBytes = kRatio * kHeadDim * 2;                      // 2048: 4 K (or V) rows
+constexpr int kUnitBytes = 2 * kHalfBytes;                             // 4096: K rows then V rows
+constexpr int kSlotStride = kUnitBytes + 32;                           // 4128: 16-B bank-group skew of 2
+constexpr int kStageBytes = kUnitsPerTile * kSlotStride;
 constexpr int kQRowStride = kHeadDim * 2 + 64;                         // 576
 constexpr int kQBufBytes = 16 * kQRowStride;
 constexpr int kCombRow = kHeadDim + 4;                                 // floats
@@ -75,8 +77,7 @@ constexpr int kBarConsumers = 1;                  // named barrier id
 constexpr uint64_t kNoCopy = ~0ull;
 
 struct DecodeArgs {
-  const __nv_bfloat16* k_pages;
-  const __nv_bfloat16* v_pages;
+  const __nv_bfloat16* kv_pages;
   const int32_t* bt;
   int32_t num_pages, max_seqs, mpps, hkv;
   const __nv_bfloat16* q;
@@ -248,10 +249,9 @@ __device__ void lookup_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int6
         if (phys < 0 || phys >= a.num_pages) {
           flag(a.st, QSA_DEV_BAD_PAGE);
         } else {
-          off = (((uint64_t)phys * a.hkv + s.g) * kPage + (uint64_t)(j % kBlocksPerPage) * kRatio) * kHeadDim;
+          off = (((uint64_t)phys * a.hkv + s.g) * kBlocksPerPage + (uint64_t)(j % kBlocksPerPage)) *
+                (2 * kRatio * kHeadDim);
           rows = (1u << nrows) - 1u;
-          prefetch_l2(a.k_pages + off, kUnitBytes);
-          prefetch_l2(a.v_pages + off, kUnitBytes);
         }
       }
     }
@@ -304,14 +304,12 @@ __device__ void copy_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
       const uint32_t ncopy = __popc(__ballot_sync(0xffffffffu, do_copy));
       if (lane == 0) {
         meta[stage] = rowmask;
-        mbar_arrive_expect_tx(bar_full + stage * 8, ncopy * 2u * kUnitBytes);
+        mbar_arrive_expect_tx(bar_full + stage * 8, ncopy * kUnitBytes);
       }
       __syncwarp();
-      if (do_copy) {
-        const uint32_t dk = ring + stage * kStageBytes + slot4 * kSlotStride;
-        bulk_g2s(dk, a.k_pages + off, kUnitBytes, bar_full + stage * 8, policy);
-        bulk_g2s(dk + kUnitsPerTile * kSlotStride, a.v_pages + off, kUnitBytes, bar_full + stage * 8, policy);
-      }
+      if (do_copy)
+        bulk_g2s(ring + stage * kStageBytes + slot4 * kSlotStride, a.kv_pages + off, kUnitBytes,
+                 bar_full + stage * 8, policy);
     }
     if (stop) break;
   }
@@ -363,10 +361,10 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
   // S/P columns held by this lane: n = 2tq + e -> (slot (tq + 2e) & 3, row 2j + e)
   const int ps0 = tq, ps1 = (tq + 2) & 3;
   // V tokens of the PV B fragment: (ps0,row0) (ps1,row1) (ps0,row2) (ps1,row3)
-  const uint32_t v_off0 = kUnitsPerTile * kSlotStride + ps0 * kSlotStride + 0 * 512 + gq * 16;
-  const uint32_t v_off1 = kUnitsPerTile * kSlotStride + ps1 * kSlotStride + 1 * 512 + gq * 16;
-  const uint32_t v_off2 = kUnitsPerTile * kSlotStride + ps0 * kSlotStride + 2 * 512 + gq * 16;
-  const uint32_t v_off3 = kUnitsPerTile * kSlotStride + ps1 * kSlotStride + 3 * 512 + gq * 16;
+  const uint32_t v_off0 = ps0 * kSlotStride + kHalfBytes + 0 * 512 + gq * 16;
+  const uint32_t v_off1 = ps1 * kSlotStride + kHalfBytes + 1 * 512 + gq * 16;
+  const uint32_t v_off2 = ps0 * kSlotStride + kHalfBytes + 2 * 512 + gq * 16;
+  const uint32_t v_off3 = ps1 * kSlotStride + kHalfBytes + 3 * 512 + gq * 16;
   const int vb0 = ps0 * 4 + 0, vb1 = ps1 * 4 + 1, vb2 = ps0 * 4 + 2, vb3 = ps1 * 4 + 3;
 
   int64_t T_base = 0;
@@ -654,16 +652,15 @@ extern "C" int qsa_sparse_decode(const qsa_cache_t* cache, const void* q, int32_
   if (hq / c.num_kv_heads > QSA_MAX_GROUP) return QSA_ERR_UNSUPPORTED;
   if (max_splits < qsa_splits_bound(k, chunk_units)) return QSA_ERR_INVALID_ARG;
   if (nq == 0) return QSA_OK;
-  if (!c.k_pages || !c.v_pages || !c.block_table || !q || !q_seq || !q_pos || !count || !part_o || !part_lse ||
+  if (!c.kv_pages || !c.block_table || !q || !q_seq || !q_pos || !count || !part_o || !part_lse ||
       (k > 0 && !sel))
     return QSA_ERR_INVALID_ARG;
   if (c.num_pages < 1 || c.max_seqs < 1 || c.max_pages_per_seq < 1) return QSA_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(c.k_pages) | reinterpret_cast<uintptr_t>(c.v_pages) |
+  if ((reinterpret_cast<uintptr_t>(c.kv_pages) |
        reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(part_o)) & 15u)
     return QSA_ERR_INVALID_ARG;
   DecodeArgs a;
-  a.k_pages = static_cast<const __nv_bfloat16*>(c.k_pages);
-  a.v_pages = static_cast<const __nv_bfloat16*>(c.v_pages);
+  a.kv_pages = static_cast<const __nv_bfloat16*>(c.kv_pages);
   a.bt = c.block_table;
   a.num_pages = c.num_pages;
   a.max_seqs = c.max_seqs;

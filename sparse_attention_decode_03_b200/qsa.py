@@ -39,7 +39,7 @@ class QSAError(RuntimeError):
 
 
 class qsa_cache_t(ctypes.Structure):
-    _fields_ = [("k_pages", ctypes.c_void_p), ("v_pages", ctypes.c_void_p), ("kc_pages", ctypes.c_void_p),
+    _fields_ = [("kv_pages", ctypes.c_void_p), ("kc_pages", ctypes.c_void_p),
                 ("kc_partial", ctypes.c_void_p), ("block_table", ctypes.c_void_p), ("num_pages", ctypes.c_int32),
                 ("max_seqs", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32)]
@@ -112,15 +112,18 @@ def _req(t: torch.Tensor, name: str, dtype, shape=None):
 
 class PagedCache:
     """Device buffers of one cache group: main K/V pages and the compressed-indexer
-    side cache, paged by the same page ids, plus the per-sequence open-block sum."""
+    side cache, paged by the same page ids, plus the per-sequence open-block sum.
+
+    kv_pages is [page][Hkv][16 micro-blocks][2 (K, V)][4 rows][256]: one selected
+    micro-block of one KV head is a contiguous 4 KiB run."""
 
     def __init__(self, num_pages: int, max_seqs: int, max_pages_per_seq: int, num_kv_heads: int,
                  block_table: torch.Tensor | None = None, device="cuda"):
         dev = torch.device(device)
         self.num_pages, self.max_seqs, self.max_pages_per_seq, self.num_kv_heads = (
             int(num_pages), int(max_seqs), int(max_pages_per_seq), int(num_kv_heads))
-        self.k_pages = torch.empty((num_pages, num_kv_heads, PAGE_TOKENS, HEAD_DIM), dtype=torch.bfloat16, device=dev)
-        self.v_pages = torch.empty_like(self.k_pages)
+        self.kv_pages = torch.empty((num_pages, num_kv_heads, BLOCKS_PER_PAGE, 2, RATIO, HEAD_DIM),
+                                    dtype=torch.bfloat16, device=dev)
         self.kc_pages = torch.empty((num_pages, BLOCKS_PER_PAGE, IDX_DIM), dtype=torch.bfloat16, device=dev)
         self.kc_partial = torch.zeros((max_seqs, IDX_DIM), dtype=torch.float32, device=dev)
         if block_table is None:
@@ -131,10 +134,17 @@ class PagedCache:
 
     def struct(self) -> qsa_cache_t:
         if self._struct is None:
-            self._struct = qsa_cache_t(self.k_pages.data_ptr(), self.v_pages.data_ptr(), self.kc_pages.data_ptr(),
+            self._struct = qsa_cache_t(self.kv_pages.data_ptr(), self.kc_pages.data_ptr(),
                                        self.kc_partial.data_ptr(), self.block_table.data_ptr(), self.num_pages,
                                        self.max_seqs, self.max_pages_per_seq, self.num_kv_heads)
         return self._struct
+
+    def k_view(self) -> torch.Tensor:
+        """K as [page][Hkv][64][256] (a strided view, for inspection)."""
+        return self.kv_pages[:, :, :, 0].reshape(self.num_pages, self.num_kv_heads, PAGE_TOKENS, HEAD_DIM)
+
+    def v_view(self) -> torch.Tensor:
+        return self.kv_pages[:, :, :, 1].reshape(self.num_pages, self.num_kv_heads, PAGE_TOKENS, HEAD_DIM)
 
     @property
     def capacity_tokens(self) -> int:
@@ -268,7 +278,7 @@ class Decoder:
 
     def __init__(self, cache: PagedCache, hq: int, max_nq: int, k: int = 512, scale: float = 1.0 / 16.0,
                  target_ctas: int | None = None, chunk_units: int | None = None, scores_ld: int | None = None):
-        dev = cache.k_pages.device
+        dev = cache.kv_pages.device
         self.cache, self.hq, self.k, self.scale, self.max_nq = cache, hq, k, scale, max_nq
         if target_ctas is None:
             target_ctas = torch.cuda.get_device_properties(dev).multi_processor_count

@@ -25,7 +25,7 @@ def test_library_exports_every_declared_symbol():
     lib = ctypes.CDLL(qsa.LIB_PATH)
     for n in header_functions():
         assert hasattr(lib, n), n
-    assert qsa.ABI_VERSION == 1
+    assert qsa.ABI_VERSION == 2
     assert qsa.status_string(0) == "QSA_OK" and qsa.status_string(-3) == "QSA_ERR_CUDA"
 
 
@@ -45,7 +45,7 @@ def test_host_validation_returns_before_any_cuda_call():
     import sparse_attention_decode_03_b200 as qsa
     L = qsa.qsa.LIB
     fake = ctypes.c_void_p(0x1000)
-    cache = qsa.qsa.qsa_cache_t(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 10, 2, 4, 2)
+    cache = qsa.qsa.qsa_cache_t(0x1000, 0x1000, 0x1000, 0x1000, 10, 2, 4, 2)
     cp = ctypes.byref(cache)
     # sparse decode: Hq not a multiple of Hkv; group too large; K too large; too few split slots
     args = lambda hq, k, chunk, ms: (cp, fake, 1, hq, fake, fake, fake, fake, k, 0.0625, chunk, ms, fake, fake, None, None)

@@ -85,8 +85,7 @@ def _append_irregular(cache, wl, st):
 def test_append_kv_bit_exact(name, lengths):
     wl = C.shrink(C.get(name), lengths, page_perm=True)
     cache = H.new_cache(wl)
-    cache.k_pages.fill_(1024.0)
-    cache.v_pages.fill_(1024.0)
+    cache.kv_pages.fill_(1024.0)
     cache.kc_pages.fill_(512.0)
     st = _status()
     _append_irregular(cache, wl, st)
@@ -96,8 +95,8 @@ def test_append_kv_bit_exact(name, lengths):
     for b, L in enumerate(wl.lengths):
         pos = torch.arange(L)
         pg, row = bt[b, pos // 64].long(), pos % 64
-        k_gpu = cache.k_pages.cpu()[pg, :, row]
-        v_gpu = cache.v_pages.cpu()[pg, :, row]
+        k_gpu = cache.k_view().cpu()[pg, :, row]
+        v_gpu = cache.v_view().cpu()[pg, :, row]
         assert torch.equal(k_gpu.view(torch.int16), C.k_rows(wl, b, pos).view(torch.int16))
         assert torch.equal(v_gpu.view(torch.int16), C.v_rows(wl, b, pos).view(torch.int16))
         kid = C.kidx_rows(wl, b, pos).float().numpy()
@@ -112,7 +111,8 @@ def test_append_kv_bit_exact(name, lengths):
         # untouched slots keep their sentinel
         last = int(bt[b, (L - 1) // 64])
         if L % 64:
-            assert torch.all(cache.k_pages[last, :, L % 64:].float() == 1024.0)
+            assert torch.all(cache.k_view()[last, :, L % 64:].float() == 1024.0)
+            assert torch.all(cache.v_view()[last, :, L % 64:].float() == 1024.0)
         if nb % 16:
             assert torch.all(cache.kc_pages[last, nb % 16:].float() == 512.0)
 
@@ -133,8 +133,10 @@ def test_append_chunking_is_bitwise_invariant():
     assert torch.equal(bits16(a.kc_pages.cpu()[bt[0, j // 16].long(), j % 16]),
                        bits16(b.kc_pages.cpu()[bt[0, j // 16].long(), j % 16]))
     assert torch.equal(a.kc_partial[0].cpu().view(torch.int32), b.kc_partial[0].cpu().view(torch.int32))
-    assert torch.equal(bits16(a.k_pages.cpu()[bt[0, pos // 64].long(), :, pos % 64]),
-                       bits16(b.k_pages.cpu()[bt[0, pos // 64].long(), :, pos % 64]))
+    assert torch.equal(bits16(a.k_view().cpu()[bt[0, pos // 64].long(), :, pos % 64]),
+                       bits16(b.k_view().cpu()[bt[0, pos // 64].long(), :, pos % 64]))
+    assert torch.equal(bits16(a.v_view().cpu()[bt[0, pos // 64].long(), :, pos % 64]),
+                       bits16(b.v_view().cpu()[bt[0, pos // 64].long(), :, pos % 64]))
 
 
 # ---------------------------------------------------------------- indexer + top-k
