@@ -25,11 +25,13 @@
 //     The bulk-copy engine costs about a hundred cycles per operation on B200,
 //     whatever its size; 4 KiB operations keep it near HBM speed where 2 KiB
 //     ones cap an SM at about two thirds of its share.
-//   consumers: tile T (16 tokens) belongs to warp T % 4; each warp runs
-//     S = Q K^T and O += P V with mma.sync m16n8k16 (M = 16 Q-head rows of the
-//     KV group, fp32 accumulate), online softmax in registers; at the end of a
-//     segment the 4 warps merge their (m, l, O) in two rounds through shared
-//     memory and write the partial.
+//   consumers: 4 pairs of warps; tile T (16 tokens) belongs to pair T % 4.
+//     Both warps of a pair compute S = Q K^T for the tile and the online
+//     softmax (mma.sync m16n8k16, M = 16 Q-head rows of the KV group, fp32
+//     accumulate); each accumulates O += P V for its half of the 256 output
+//     dims, which halves the accumulator registers and lets 8 consumer warps
+//     keep the copies fed.  At the end of a segment the 4 pairs merge their
+//     (m, l, O) in two rounds through shared memory and write the partial.
 // Shared-memory layouts are skewed so that every 16-byte fragment read is
 // bank-conflict free (micro-block slots 4128 B apart, Q rows 576 B apart).
 #include "qsa_common.cuh"
@@ -38,13 +40,14 @@ namespace {
 
 using namespace qsa;
 
-constexpr int kConsumerWarps = 4;
-constexpr int kCopyWarp = kConsumerWarps;         // warp 4
-constexpr int kLookupWarp = kConsumerWarps + 1;   // warp 5
+constexpr int kConsumerWarps = 8;                 // 4 pairs
+constexpr int kPairs = kConsumerWarps / 2;
+constexpr int kCopyWarp = kConsumerWarps;         // warp 8
+constexpr int kLookupWarp = kConsumerWarps + 1;   // warp 9
 constexpr int kThreads = (kConsumerWarps + 2) * 32;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 // A stage is reused by tile T + kStages; with kStages a multiple of the consumer
-// warp count and tile T owned by warp T % 4, that tile's owner is the warp that
+// pair count and tile T owned by pair T % 4, that tile's owner is the pair that
 // consumed tile T, so no mbarrier wait can ever skip a phase (a parity wait can
 // only name the current phase or the one before it).
 constexpr int kStages = 8;
@@ -63,7 +66,7 @@ constexpr int kOffRing = 0;
 constexpr int kOffQ = kOffRing + kStages * kStageBytes;
 constexpr int kOffComb = kOffQ + kQBufBytes;
 constexpr int kOffML = kOffComb + kCombBytes;
-constexpr int kOffDescOff = kOffML + kConsumerWarps * 16 * 2 * 4;
+constexpr int kOffDescOff = kOffML + kPairs * 16 * 2 * 4;
 constexpr int kOffDescRows = kOffDescOff + kDescSlots * kBatch * 8;
 constexpr int kOffMeta = kOffDescRows + kDescSlots * kBatch * 4;
 constexpr int kOffBar = (kOffMeta + kStages * 4 + 7) & ~7;
@@ -71,7 +74,7 @@ constexpr int kNumBars = 2 * kStages + 2 * kDescSlots;
 constexpr int kOffAbort = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffAbort + 16;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kStages % kConsumerWarps == 0, "tile ownership must repeat with the stage ring");
+static_assert(kStages % kPairs == 0, "tile ownership must repeat with the stage ring");
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr int kBarConsumers = 1;                  // named barrier id
 constexpr uint64_t kNoCopy = ~0ull;
@@ -341,8 +344,10 @@ __device__ __forceinline__ bool consumer_wait(const DecodeArgs& a, uint32_t bar,
 }
 
 __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_t x1) {
-  const int tid = threadIdx.x;  // 0..127
+  const int tid = threadIdx.x;  // 0..255
   const int warp = tid >> 5, lane = tid & 31;
+  const int cp = warp >> 1;     // consumer pair: owns tiles T with T % 4 == cp
+  const int half = warp & 1;    // output dims [128 * half, 128 * half + 128)
   const int gq = lane >> 2, tq = lane & 3;
   const uint32_t ring = smem_u32(smem + kOffRing);
   const uint32_t bar_full = smem_u32(smem + kOffBar);
@@ -360,19 +365,19 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
   const uint32_t k_off = ks * kSlotStride + ke * 512 + tq * 16;
   // S/P columns held by this lane: n = 2tq + e -> (slot (tq + 2e) & 3, row 2j + e)
   const int ps0 = tq, ps1 = (tq + 2) & 3;
-  // V tokens of the PV B fragment: (ps0,row0) (ps1,row1) (ps0,row2) (ps1,row3)
-  const uint32_t v_off0 = ps0 * kSlotStride + kHalfBytes + 0 * 512 + gq * 16;
-  const uint32_t v_off1 = ps1 * kSlotStride + kHalfBytes + 1 * 512 + gq * 16;
-  const uint32_t v_off2 = ps0 * kSlotStride + kHalfBytes + 2 * 512 + gq * 16;
-  const uint32_t v_off3 = ps1 * kSlotStride + kHalfBytes + 3 * 512 + gq * 16;
+  // V tokens of the PV B fragment: (ps0,row0) (ps1,row1) (ps0,row2) (ps1,row3); this
+  // warp reads V chunks 8qq + gq for qq in {2 half, 2 half + 1}
+  const uint32_t vh = kHalfBytes + half * 256;
+  const uint32_t v_off0 = ps0 * kSlotStride + vh + 0 * 512 + gq * 16;
+  const uint32_t v_off1 = ps1 * kSlotStride + vh + 1 * 512 + gq * 16;
+  const uint32_t v_off2 = ps0 * kSlotStride + vh + 2 * 512 + gq * 16;
+  const uint32_t v_off3 = ps1 * kSlotStride + vh + 3 * 512 + gq * 16;
   const int vb0 = ps0 * 4 + 0, vb1 = ps1 * 4 + 1, vb2 = ps0 * 4 + 2, vb3 = ps1 * 4 + 3;
 
   int64_t T_base = 0;
-  int seg_idx = 0;
-  for (int64_t pair = x0 / n_slots; pair <= (x1 - 1) / n_slots; ++pair, ++seg_idx) {
+  for (int64_t pair = x0 / n_slots; pair <= (x1 - 1) / n_slots; ++pair) {
     const Seg s = make_seg(a, pair, x0, x1, tid == 0);
-    uint8_t* qbuf = smem + kOffQ;  // the merge barriers of the last segment order reuse
-    const uint32_t qb = smem_u32(qbuf);
+    const uint32_t qb = smem_u32(smem + kOffQ);  // the merge barriers of the last segment order reuse
     // ---- stage Q rows of this KV group (rows >= G are zero)
     for (int idx = tid; idx < 16 * 32; idx += kConsumerThreads) {
       const int row = idx >> 5, c = idx & 31;
@@ -384,13 +389,13 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
     named_bar_sync(kBarConsumers, kConsumerThreads);
 
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    float o[32][4];
+    float o[16][4];
 #pragma unroll
-    for (int nt = 0; nt < 32; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+    for (int nt = 0; nt < 16; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
 
-    // tile T (counted over the whole chunk) belongs to warp T % 4
-    const int first_ti = (int)(((int64_t)warp - T_base % kConsumerWarps + kConsumerWarps) % kConsumerWarps);
-    for (int ti = first_ti; ti < s.n_tiles; ti += kConsumerWarps) {
+    // tile T (counted over the whole chunk) belongs to pair T % 4
+    const int first_ti = (int)(((int64_t)cp - T_base % kPairs + kPairs) % kPairs);
+    for (int ti = first_ti; ti < s.n_tiles; ti += kPairs) {
       const int64_t T = T_base + ti;
       const int stage = (int)(T % kStages);
       if (!*abort_flag) consumer_wait(a, bar_full + stage * 8, (uint32_t)((T / kStages) & 1), abort_flag);
@@ -398,7 +403,7 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
       const uint32_t mask = meta[stage];
       const uint32_t kb = ring + stage * kStageBytes;
 
-      // ---- S = Q K^T : two n-tiles of 8 tokens, k = 256 dims in 16 steps
+      // ---- S = Q K^T : two n-tiles of 8 tokens, k = 256 dims in 16 steps (both warps of the pair)
       float sa[2][4], sb[2][4];
 #pragma unroll
       for (int j = 0; j < 2; ++j)
@@ -452,7 +457,7 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
       l1 = l1 * al1 + ((pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]));
       if (al0 != 1.f || al1 != 1.f) {
 #pragma unroll
-        for (int nt = 0; nt < 32; ++nt) {
+        for (int nt = 0; nt < 16; ++nt) {
           o[nt][0] *= al0;
           o[nt][1] *= al0;
           o[nt][2] *= al1;
@@ -467,16 +472,16 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
       split_bf16(pr[1][0], pr[1][1], pa[2], pl[2]);
       split_bf16(pr[1][2], pr[1][3], pa[3], pl[3]);
 
-      // ---- O += P V : 32 n-tiles over the 256 output dims, k = the tile's 16 tokens
+      // ---- O += P V for this warp's 128 dims: 16 n-tiles, k = the tile's 16 tokens
       const bool full = mask == 0xffffu;
       const bool ok0 = (mask >> vb0) & 1u, ok1 = (mask >> vb1) & 1u;
       const bool ok2 = (mask >> vb2) & 1u, ok3 = (mask >> vb3) & 1u;
 #pragma unroll
-      for (int qq = 0; qq < 4; ++qq) {
-        uint4 x0v = lds128(kb + v_off0 + qq * 128);
-        uint4 x1v = lds128(kb + v_off1 + qq * 128);
-        uint4 x2v = lds128(kb + v_off2 + qq * 128);
-        uint4 x3v = lds128(kb + v_off3 + qq * 128);
+      for (int qh = 0; qh < 2; ++qh) {
+        uint4 x0v = lds128(kb + v_off0 + qh * 128);
+        uint4 x1v = lds128(kb + v_off1 + qh * 128);
+        uint4 x2v = lds128(kb + v_off2 + qh * 128);
+        uint4 x3v = lds128(kb + v_off3 + qh * 128);
         if (!full) {  // masked rows may hold stale or never-written data
           if (!ok0) x0v = make_uint4(0, 0, 0, 0);
           if (!ok1) x1v = make_uint4(0, 0, 0, 0);
@@ -493,104 +498,104 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
           const uint32_t hi01 = __byte_perm(a0[r], a1[r], 0x7632);
           const uint32_t lo23 = __byte_perm(a2[r], a3[r], 0x5410);
           const uint32_t hi23 = __byte_perm(a2[r], a3[r], 0x7632);
-          mma_bf16_16816(o[qq * 8 + 2 * r], pa[0], pa[1], pa[2], pa[3], lo01, lo23);
-          mma_bf16_16816(o[qq * 8 + 2 * r], pl[0], pl[1], pl[2], pl[3], lo01, lo23);
-          mma_bf16_16816(o[qq * 8 + 2 * r + 1], pa[0], pa[1], pa[2], pa[3], hi01, hi23);
-          mma_bf16_16816(o[qq * 8 + 2 * r + 1], pl[0], pl[1], pl[2], pl[3], hi01, hi23);
+          mma_bf16_16816(o[qh * 8 + 2 * r], pa[0], pa[1], pa[2], pa[3], lo01, lo23);
+          mma_bf16_16816(o[qh * 8 + 2 * r + 1], pa[0], pa[1], pa[2], pa[3], hi01, hi23);
+          mma_bf16_16816(o[qh * 8 + 2 * r], pl[0], pl[1], pl[2], pl[3], lo01, lo23);
+          mma_bf16_16816(o[qh * 8 + 2 * r + 1], pl[0], pl[1], pl[2], pl[3], hi01, hi23);
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_empty + stage * 8);
+      if (lane == 0) mbar_arrive(bar_empty + stage * 8);  // both warps of the pair arrive
     }
     T_base += s.n_tiles;
 
-    // ---- merge the 4 warps' (m, l, O) and write the split partial
+    // ---- merge the 4 pairs' (m, l, O) and write the split partial
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    if (tq == 0) {
-      ml[(warp * 16 + gq) * 2 + 0] = m0;
-      ml[(warp * 16 + gq) * 2 + 1] = l0;
-      ml[(warp * 16 + gq + 8) * 2 + 0] = m1;
-      ml[(warp * 16 + gq + 8) * 2 + 1] = l1;
+    if (half == 0 && tq == 0) {  // both warps of a pair hold the same m and l
+      ml[(cp * 16 + gq) * 2 + 0] = m0;
+      ml[(cp * 16 + gq) * 2 + 1] = l0;
+      ml[(cp * 16 + gq + 8) * 2 + 0] = m1;
+      ml[(cp * 16 + gq + 8) * 2 + 1] = l1;
     }
     named_bar_sync(kBarConsumers, kConsumerThreads);
-    // this warp's weight for rows gq / gq+8, and the merged lse of those rows
+    // this pair's weight for rows gq / gq+8, and the merged lse of those rows
     float fac[2], lse_row[2];
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int row = gq + 8 * half;
-      const float mine = half ? m1 : m0;
+    for (int hr = 0; hr < 2; ++hr) {
+      const int row = gq + 8 * hr;
+      const float mine = hr ? m1 : m0;
       float M = -INFINITY;
-      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ml[(w * 16 + row) * 2]);
-      fac[half] = 0.f;
-      lse_row[half] = -INFINITY;
+      for (int w = 0; w < kPairs; ++w) M = fmaxf(M, ml[(w * 16 + row) * 2]);
+      fac[hr] = 0.f;
+      lse_row[hr] = -INFINITY;
       if (M != -INFINITY) {
         float L = 0.f;
-        for (int w = 0; w < kConsumerWarps; ++w) {
+        for (int w = 0; w < kPairs; ++w) {
           const float mw = ml[(w * 16 + row) * 2];
           if (mw != -INFINITY) L += ml[(w * 16 + row) * 2 + 1] * exp2f(mw - M);
         }
-        fac[half] = mine != -INFINITY ? exp2f(mine - M) / L : 0.f;
-        lse_row[half] = (M + log2f(L)) * 0.69314718055994530942f;
+        fac[hr] = mine != -INFINITY ? exp2f(mine - M) / L : 0.f;
+        lse_row[hr] = (M + log2f(L)) * 0.69314718055994530942f;
       }
     }
 #pragma unroll
-    for (int nt = 0; nt < 32; ++nt) {
+    for (int nt = 0; nt < 16; ++nt) {
       o[nt][0] *= fac[0];
       o[nt][1] *= fac[0];
       o[nt][2] *= fac[1];
       o[nt][3] *= fac[1];
     }
-    // n-tile 8qq + w8 holds dims 64qq + 16tq + w8 (c0/c2) and 64qq + 16tq + 8 + w8 (c1/c3)
+    // local n-tile 8qh + w8 holds dims 128half + 64qh + 16tq + w8 (c0/c2) and + 8 (c1/c3)
     auto store_rows = [&](float* base, int row_stride) {
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int row = gq + 8 * half;
+      for (int hr = 0; hr < 2; ++hr) {
+        const int row = gq + 8 * hr;
         if (row >= G) continue;
-        const int c = 2 * half;
+        const int c = 2 * hr;
 #pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-          float4* d4 = reinterpret_cast<float4*>(base + (size_t)row * row_stride + 64 * qq + 16 * tq);
-          d4[0] = make_float4(o[qq * 8 + 0][c], o[qq * 8 + 1][c], o[qq * 8 + 2][c], o[qq * 8 + 3][c]);
-          d4[1] = make_float4(o[qq * 8 + 4][c], o[qq * 8 + 5][c], o[qq * 8 + 6][c], o[qq * 8 + 7][c]);
-          d4[2] = make_float4(o[qq * 8 + 0][c + 1], o[qq * 8 + 1][c + 1], o[qq * 8 + 2][c + 1], o[qq * 8 + 3][c + 1]);
-          d4[3] = make_float4(o[qq * 8 + 4][c + 1], o[qq * 8 + 5][c + 1], o[qq * 8 + 6][c + 1], o[qq * 8 + 7][c + 1]);
+        for (int qh = 0; qh < 2; ++qh) {
+          float4* d4 = reinterpret_cast<float4*>(base + (size_t)row * row_stride + 128 * half + 64 * qh + 16 * tq);
+          d4[0] = make_float4(o[qh * 8 + 0][c], o[qh * 8 + 1][c], o[qh * 8 + 2][c], o[qh * 8 + 3][c]);
+          d4[1] = make_float4(o[qh * 8 + 4][c], o[qh * 8 + 5][c], o[qh * 8 + 6][c], o[qh * 8 + 7][c]);
+          d4[2] = make_float4(o[qh * 8 + 0][c + 1], o[qh * 8 + 1][c + 1], o[qh * 8 + 2][c + 1], o[qh * 8 + 3][c + 1]);
+          d4[3] = make_float4(o[qh * 8 + 4][c + 1], o[qh * 8 + 5][c + 1], o[qh * 8 + 6][c + 1], o[qh * 8 + 7][c + 1]);
         }
       }
     };
     auto add_rows = [&](const float* base) {
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int row = gq + 8 * half;
+      for (int hr = 0; hr < 2; ++hr) {
+        const int row = gq + 8 * hr;
         if (row >= G) continue;
-        const int c = 2 * half;
+        const int c = 2 * hr;
 #pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-          const float4* s4 = reinterpret_cast<const float4*>(base + row * kCombRow + 64 * qq + 16 * tq);
+        for (int qh = 0; qh < 2; ++qh) {
+          const float4* s4 = reinterpret_cast<const float4*>(base + row * kCombRow + 128 * half + 64 * qh + 16 * tq);
           const float4 x0 = s4[0], x1 = s4[1], x2 = s4[2], x3 = s4[3];
-          o[qq * 8 + 0][c] += x0.x; o[qq * 8 + 1][c] += x0.y; o[qq * 8 + 2][c] += x0.z; o[qq * 8 + 3][c] += x0.w;
-          o[qq * 8 + 4][c] += x1.x; o[qq * 8 + 5][c] += x1.y; o[qq * 8 + 6][c] += x1.z; o[qq * 8 + 7][c] += x1.w;
-          o[qq * 8 + 0][c + 1] += x2.x; o[qq * 8 + 1][c + 1] += x2.y; o[qq * 8 + 2][c + 1] += x2.z;
-          o[qq * 8 + 3][c + 1] += x2.w;
-          o[qq * 8 + 4][c + 1] += x3.x; o[qq * 8 + 5][c + 1] += x3.y; o[qq * 8 + 6][c + 1] += x3.z;
-          o[qq * 8 + 7][c + 1] += x3.w;
+          o[qh * 8 + 0][c] += x0.x; o[qh * 8 + 1][c] += x0.y; o[qh * 8 + 2][c] += x0.z; o[qh * 8 + 3][c] += x0.w;
+          o[qh * 8 + 4][c] += x1.x; o[qh * 8 + 5][c] += x1.y; o[qh * 8 + 6][c] += x1.z; o[qh * 8 + 7][c] += x1.w;
+          o[qh * 8 + 0][c + 1] += x2.x; o[qh * 8 + 1][c + 1] += x2.y; o[qh * 8 + 2][c + 1] += x2.z;
+          o[qh * 8 + 3][c + 1] += x2.w;
+          o[qh * 8 + 4][c + 1] += x3.x; o[qh * 8 + 5][c + 1] += x3.y; o[qh * 8 + 6][c + 1] += x3.z;
+          o[qh * 8 + 7][c + 1] += x3.w;
         }
       }
     };
-    // round 1: warps 2, 3 hand their O to warps 0, 1; round 2: warp 1 to warp 0
-    if (warp >= 2) store_rows(comb + (warp - 2) * 16 * kCombRow, kCombRow);
+    // round 1: pairs 2, 3 hand their O to pairs 0, 1; round 2: pair 1 to pair 0
+    if (cp >= 2) store_rows(comb + (cp - 2) * 16 * kCombRow, kCombRow);
     named_bar_sync(kBarConsumers, kConsumerThreads);
-    if (warp < 2) add_rows(comb + warp * 16 * kCombRow);
+    if (cp < 2) add_rows(comb + cp * 16 * kCombRow);
     named_bar_sync(kBarConsumers, kConsumerThreads);
-    if (warp == 1) store_rows(comb, kCombRow);
+    if (cp == 1) store_rows(comb, kCombRow);
     named_bar_sync(kBarConsumers, kConsumerThreads);
     const size_t row0 = ((size_t)s.q * a.max_splits + s.split) * a.hq + (size_t)s.g * G;
-    if (warp == 0) {
+    if (cp == 0) {
       add_rows(comb);
       store_rows(a.part_o + row0 * kHeadDim, kHeadDim);
-      if (tq == 0) {
+      if (half == 0 && tq == 0) {
         if (gq < G) a.part_lse[row0 + gq] = lse_row[0];
         if (gq + 8 < G) a.part_lse[row0 + gq + 8] = lse_row[1];
       }
@@ -615,7 +620,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(DecodeArgs a
     const uint32_t bf = smem_u32(smem + kOffBar);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(bf + i * 8, 1);                  // full: copy warp's arrive + tx bytes
-      mbar_init(bf + (kStages + i) * 8, 1);      // empty: one consumer warp
+      mbar_init(bf + (kStages + i) * 8, 2);      // empty: both warps of the owning pair
     }
     for (int i = 0; i < kDescSlots; ++i) {
       mbar_init(bf + (2 * kStages + i) * 8, 1);               // descriptors written (lookup warp)

@@ -6,25 +6,28 @@
 // the tie-break (lower index first) and ascending output order are the fixed
 // readings.
 //
-// One CTA per query, order-preserving uint32 keys of the fp32 scores.
-// Common path (rows up to 65,536 blocks): ONE vectorised read of the scores
-// (L2-resident), then shared memory.
-//   1. read the row once: keep every key's high 16 bits in shared memory and
-//      the row's min / max key;
+// Order-preserving uint32 keys of the fp32 scores.  One thread-block cluster
+// of 8 CTAs per query (decode batches have only 32-64 queries, so a single CTA
+// per query leaves the per-key work on too few SMs).  CTA r of the cluster owns
+// the r-th contiguous eighth of the row and keeps its keys in shared memory
+// after one vectorised read.  Then:
+//   1. cluster-wide min / max key (distributed shared memory);
 //   2. radix select with adaptive 11-bit windows starting at the highest bit
-//      where the keys differ (scores share their top exponent bits, so fixed
-//      top-bit bins would all land in a couple of bins): each window is a
-//      shared-memory histogram of the keys that still match the prefix; bits
-//      below 16 are fetched from L2 for those keys only.  The result is the
-//      exact K-th largest key T;
-//   3. a word-wise ballot pass writes a bitmap of keys > T and counts keys == T
-//      per 32 indices; a block scan ranks the ties in index order and the
-//      lowest-index ones are added;
-//   4. the K indices are emitted in ascending order from the bitmap.
-// Longer rows take the general path: three radix passes over the scores
-// (12 + 12 + 8 bits) and an ordered compaction with warp ballots.
+//      where the keys differ (scores share their top exponent bits): every CTA
+//      histograms its slice, the 8 histograms are summed through distributed
+//      shared memory, and each CTA finds the same bin; this yields the exact
+//      K-th largest key T;
+//   3. each CTA ranks its keys == T in index order (word ballots, a block scan
+//      and the counts of the lower-ranked CTAs) and keeps the lowest-index
+//      ones, then writes its selected indices, in ascending order, at the
+//      offset given by the lower-ranked CTAs' counts.
+// Rows longer than 65,536 blocks take the general path in the cluster's first
+// CTA: three radix passes over the scores (12 + 12 + 8 bits) and an ordered
+// compaction with warp ballots.
 // Integer counters only: the result does not depend on atomic order.
 #include "qsa_common.cuh"
+
+#include <cooperative_groups.h>
 
 namespace {
 
@@ -79,9 +82,14 @@ __device__ void find_bin(const uint32_t* hist, int nbins, uint32_t remaining, ui
   __syncthreads();
 }
 
-constexpr int kMaxFast = 65536;          // blocks per query on the shared-memory path
+constexpr int kCluster = 8;                    // CTAs per query
+constexpr int kCThreads = 512;                 // threads per cluster CTA
+constexpr int kCWarps = kCThreads / 32;
+constexpr int kSliceCap = 8192;                // keys per CTA on the cluster path
+constexpr int kMaxFast = kCluster * kSliceCap; // 65,536 blocks per query
 constexpr int kUnroll = 8;
-constexpr int kWin = 11;                 // radix window bits
+constexpr int kWin = 11;                       // radix window bits
+constexpr int kWinBins = 1 << kWin;
 
 __device__ __forceinline__ void load_keys(const float* s, int i0, int n, uint32_t (&key)[kUnroll]) {
 #pragma unroll
@@ -89,50 +97,6 @@ __device__ __forceinline__ void load_keys(const float* s, int i0, int n, uint32_
     const int i = i0 + u * kThreads;
     key[u] = i < n ? float_key(s[i]) : 0u;
   }
-}
-
-// Shared-memory histogram increment.  A warp whose live lanes all hit one bin
-// (common when scores crowd together) adds once; otherwise per-lane atomics.
-__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool live) {
-  const uint32_t act = __ballot_sync(0xffffffffu, live);
-  if (act == 0) return;
-  const int leader = __ffs(act) - 1;
-  const uint32_t b0 = __shfl_sync(0xffffffffu, bin, leader);
-  if (__all_sync(0xffffffffu, !live || bin == b0)) {
-    if ((threadIdx.x & 31) == leader) atomicAdd(&hist[b0], (uint32_t)__popc(act));
-  } else if (live) {
-    atomicAdd(&hist[bin], 1u);
-  }
-}
-
-// In-place exclusive scan of v[0..m) (m <= 4 * kThreads), block-wide.
-__device__ void block_exclusive_scan(uint32_t* v, int m, uint32_t* wsum) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int per = (m + kThreads - 1) / kThreads;
-  const int lo = tid * per;
-  uint32_t loc[4] = {0, 0, 0, 0};
-  uint32_t sum = 0;
-  for (int k = 0; k < per; ++k)
-    if (lo + k < m) {
-      loc[k] = v[lo + k];
-      sum += loc[k];
-    }
-  uint32_t inc = sum;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const uint32_t x = __shfl_up_sync(0xffffffffu, inc, d);
-    if (lane >= d) inc += x;
-  }
-  if (lane == 31) wsum[warp] = inc;
-  __syncthreads();
-  uint32_t base = inc - sum;
-  for (int w = 0; w < warp; ++w) base += wsum[w];
-  for (int k = 0; k < per; ++k)
-    if (lo + k < m) {
-      v[lo + k] = base;
-      base += loc[k];
-    }
-  __syncthreads();
 }
 
 // General path: exact K-th key by three radix passes, then ordered compaction.
@@ -202,183 +166,282 @@ __device__ void topk_general(const float* s, int n, int K, int32_t* out, uint32_
   }
 }
 
-__global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  __shared__ uint32_t hist[4096];
-  __shared__ uint32_t wsum[kWarps];
-  __shared__ uint32_t wgt[kWarps], weq[kWarps];
-  __shared__ uint32_t wmin[kWarps], wmax[kWarps];
+// Shared-memory histogram increment.  A warp whose live lanes all hit one bin
+// (common when scores crowd together) adds once; otherwise per-lane atomics.
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool live) {
+  const uint32_t act = __ballot_sync(0xffffffffu, live);
+  if (act == 0) return;
+  const int leader = __ffs(act) - 1;
+  const uint32_t b0 = __shfl_sync(0xffffffffu, bin, leader);
+  if (__all_sync(0xffffffffu, !live || bin == b0)) {
+    if ((threadIdx.x & 31) == leader) atomicAdd(&hist[b0], (uint32_t)__popc(act));
+  } else if (live) {
+    atomicAdd(&hist[bin], 1u);
+  }
+}
+
+// Bin b of a merged histogram (every thread returns the same) with
+// sum_{i > b} hist[i] < remaining <= sum_{i >= b} hist[i]; *above = sum_{i > b}.
+__device__ int cluster_find_bin(const uint32_t* hist, int nbins, uint32_t remaining, uint32_t* wsum, int* s_bin,
+                                uint32_t* s_above, uint32_t* above) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (nbins + kCThreads - 1) / kCThreads;
+  const int lo = tid * per;
+  uint32_t local = 0;
+  for (int i = 0; i < per; ++i)
+    if (lo + i < nbins) local += hist[lo + i];
+  uint32_t suf = local;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const uint32_t v = __shfl_down_sync(0xffffffffu, suf, d);
+    if (lane + d < 32) suf += v;
+  }
+  if (lane == 0) wsum[warp] = suf;
+  __syncthreads();
+  uint32_t cum = suf - local;
+  for (int w = warp + 1; w < kCWarps; ++w) cum += wsum[w];
+  for (int i = per - 1; i >= 0; --i) {
+    if (lo + i >= nbins) continue;
+    const uint32_t h = hist[lo + i];
+    if (cum < remaining && remaining <= cum + h) {
+      *s_bin = lo + i;
+      *s_above = cum;
+    }
+    cum += h;
+  }
+  __syncthreads();
+  *above = *s_above;
+  return *s_bin;
+}
+
+// Block-wide exclusive prefix of one value per thread; returns the block total.
+__device__ uint32_t block_exclusive(uint32_t v, uint32_t* wsum, uint32_t* prefix) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t inc = v;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const uint32_t x = __shfl_up_sync(0xffffffffu, inc, d);
+    if (lane >= d) inc += x;
+  }
+  if (lane == 31) wsum[warp] = inc;
+  __syncthreads();
+  uint32_t base = inc - v, total = 0;
+  for (int w = 0; w < kCWarps; ++w) {
+    if (w < warp) base += wsum[w];
+    total += wsum[w];
+  }
+  __syncthreads();
+  *prefix = base;
+  return total;
+}
+
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kCThreads) topk_kernel(TopkArgs a) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ __align__(16) uint32_t keys[];  // [kSliceCap] this CTA's slice of keys (dynamic)
+  __shared__ uint32_t hist[kWinBins];    // this slice's histogram
+  __shared__ uint32_t merged[kWinBins];  // the cluster's histogram (written by all 8 CTAs)
+  __shared__ uint32_t wgt_cnt[kSliceCap / 32], weq_cnt[kSliceCap / 32];
+  __shared__ uint32_t wsum[kCWarps];
+  __shared__ uint32_t pub[4];  // published per CTA: min key, max key, #keys > T, #keys == T
   __shared__ int s_bin;
   __shared__ uint32_t s_above;
 
-  const int q = blockIdx.x;
+  const int rank = (int)cluster.block_rank();
+  const int q = blockIdx.x / kCluster;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t lt = (1u << lane) - 1u;
   const int p = a.q_pos[q];
   int64_t nb = p >= 0 ? (int64_t)(p + 1) / kRatio : 0;
-  if (p < 0 && tid == 0) flag(a.st, QSA_DEV_BAD_POS);
+  if (rank == 0 && tid == 0 && p < 0) flag(a.st, QSA_DEV_BAD_POS);
   if (nb > a.ld) {
-    if (tid == 0) flag(a.st, QSA_DEV_SCORES_LD);
+    if (rank == 0 && tid == 0) flag(a.st, QSA_DEV_SCORES_LD);
     nb = a.ld;
   }
   const int K = a.K;
   int32_t* out = a.sel + (size_t)q * K;
+  // uniform early exits (every CTA of the cluster takes the same branch, before any cluster barrier)
   if (K == 0) {
-    if (tid == 0) a.count[q] = 0;
+    if (rank == 0 && tid == 0) a.count[q] = 0;
     return;
   }
   if (nb <= K) {  // every visible block is kept
-    for (int i = tid; i < K; i += kThreads) out[i] = i < nb ? i : -1;
-    if (tid == 0) a.count[q] = (int32_t)nb;
+    if (rank == 0) {
+      for (int i = tid; i < K; i += kCThreads) out[i] = i < nb ? i : -1;
+      if (tid == 0) a.count[q] = (int32_t)nb;
+    }
     return;
   }
   const int n = (int)nb;
   const float* s = a.scores + (size_t)q * a.ld;
-  if (tid == 0) a.count[q] = K;
-  if (n > a.fast_cap) {
-    topk_general(s, n, K, out, hist, wsum, wgt, weq, &s_bin, &s_above);
+  if (n > kMaxFast) {  // selection written by topk_long_kernel, launched after this one
+    if (rank == 0 && tid == 0) a.count[q] = K;
     return;
   }
-  const int words = (n + 31) >> 5;
-  uint16_t* hi16 = reinterpret_cast<uint16_t*>(smem);                             // [fast_cap]
-  uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + (size_t)a.fast_cap * 2);  // [fast_cap / 32]
-  uint32_t* wcnt = bitmap + a.fast_cap / 32;                                       // [fast_cap / 32]
-
-  // ---- 1. one read of the row: high halves to shared memory, min / max key
+  if (rank == 0 && tid == 0) a.count[q] = K;
+  // ---- slice of this CTA: [lo, hi)
+  const int per_cta = (n + kCluster - 1) / kCluster;
+  const int lo = min(n, rank * per_cta), hi = min(n, lo + per_cta);
+  const int m = hi - lo;
   uint32_t kmin = 0xffffffffu, kmax = 0u;
-  if ((reinterpret_cast<uintptr_t>(s) & 15u) == 0) {
-    const int n4 = n >> 2;
-    const float4* s4 = reinterpret_cast<const float4*>(s);
-    constexpr int kU4 = 4;
-    for (int j0 = tid; j0 < n4; j0 += kThreads * kU4) {
-      float4 v[kU4];
+  for (int i0 = tid; i0 < m; i0 += kCThreads * kUnroll) {  // kUnroll independent loads in flight
+    uint32_t kv[kUnroll];
 #pragma unroll
-      for (int u = 0; u < kU4; ++u)
-        if (j0 + u * kThreads < n4) v[u] = __ldg(s4 + j0 + u * kThreads);
+    for (int u = 0; u < kUnroll; ++u) {
+      const int i = i0 + u * kCThreads;
+      kv[u] = i < m ? float_key(__ldg(s + lo + i)) : 0u;
+    }
 #pragma unroll
-      for (int u = 0; u < kU4; ++u) {
-        const int j = j0 + u * kThreads;
-        if (j >= n4) continue;
-        const uint32_t k0 = float_key(v[u].x), k1 = float_key(v[u].y), k2 = float_key(v[u].z), k3 = float_key(v[u].w);
-        kmin = min(kmin, min(min(k0, k1), min(k2, k3)));
-        kmax = max(kmax, max(max(k0, k1), max(k2, k3)));
-        uint2 h;
-        h.x = (k0 >> 16) | (k1 & 0xffff0000u);
-        h.y = (k2 >> 16) | (k3 & 0xffff0000u);
-        *reinterpret_cast<uint2*>(hi16 + 4 * j) = h;
+    for (int u = 0; u < kUnroll; ++u) {
+      const int i = i0 + u * kCThreads;
+      if (i < m) {
+        keys[i] = kv[u];
+        kmin = min(kmin, kv[u]);
+        kmax = max(kmax, kv[u]);
       }
-    }
-    for (int i = (n4 << 2) + tid; i < n; i += kThreads) {
-      const uint32_t k = float_key(s[i]);
-      kmin = min(kmin, k);
-      kmax = max(kmax, k);
-      hi16[i] = (uint16_t)(k >> 16);
-    }
-  } else {
-    for (int i = tid; i < n; i += kThreads) {
-      const uint32_t k = float_key(s[i]);
-      kmin = min(kmin, k);
-      kmax = max(kmax, k);
-      hi16[i] = (uint16_t)(k >> 16);
     }
   }
   kmin = __reduce_min_sync(0xffffffffu, kmin);
   kmax = __reduce_max_sync(0xffffffffu, kmax);
   if (lane == 0) {
-    wmin[warp] = kmin;
-    wmax[warp] = kmax;
+    wsum[warp] = kmin;
+    hist[warp] = kmax;
   }
   __syncthreads();
+  if (tid == 0) {
+    uint32_t mn = 0xffffffffu, mx = 0u;
+    for (int w = 0; w < kCWarps; ++w) {
+      mn = min(mn, wsum[w]);
+      mx = max(mx, hist[w]);
+    }
+    pub[0] = mn;
+    pub[1] = mx;
+  }
+  cluster.sync();
   kmin = 0xffffffffu;
   kmax = 0u;
-  for (int w = 0; w < kWarps; ++w) {
-    kmin = min(kmin, wmin[w]);
-    kmax = max(kmax, wmax[w]);
+  for (int r = 0; r < kCluster; ++r) {
+    const uint32_t* rp = cluster.map_shared_rank(pub, r);
+    kmin = min(kmin, rp[0]);
+    kmax = max(kmax, rp[1]);
   }
-  // ---- 2. radix select over the bits where the keys differ
+  // ---- radix select over the bits where the keys differ
   uint32_t prefix = kmin, remaining = (uint32_t)K;
-  int hb = kmin == kmax ? -1 : 31 - __clz(kmin ^ kmax);  // highest differing bit
-  if (hb >= 0) prefix &= ~((2u << hb) - 1u);               // (2u << 31) wraps to 0: all bits cleared
+  int hb = kmin == kmax ? -1 : 31 - __clz(kmin ^ kmax);
+  if (hb >= 0) prefix &= (hb >= 31) ? 0u : ~((2u << hb) - 1u);
   while (hb >= 0) {
-    const int lo = hb >= kWin - 1 ? hb - (kWin - 1) : 0;
-    const uint32_t nbins = 1u << (hb - lo + 1);
-    const uint32_t hmask = (hb >= 31) ? 0u : ~((2u << hb) - 1u);  // bits above the window
-    for (int i = tid; i < (int)nbins; i += kThreads) hist[i] = 0;
+    const int wlo = hb >= kWin - 1 ? hb - (kWin - 1) : 0;
+    const uint32_t nbins = 1u << (hb - wlo + 1);
+    const uint32_t hmask = (hb >= 31) ? 0u : ~((2u << hb) - 1u);
+    for (int i = tid; i < (int)nbins; i += kCThreads) hist[i] = 0;
     __syncthreads();
-    if (lo >= 16) {  // window inside the high halves: shared memory only
-      for (int i0 = tid; i0 < ((n + 31) & ~31); i0 += kThreads) {
-        const bool live0 = i0 < n;
-        const uint32_t key = live0 ? ((uint32_t)hi16[i0] << 16) : 0u;
-        const bool live = live0 && (key & hmask) == (prefix & hmask);
-        hist_add(hist, (key >> lo) & (nbins - 1), live);
+    for (int i0 = tid; i0 < ((m + 31) & ~31); i0 += kCThreads) {
+      const bool live0 = i0 < m;
+      const uint32_t key = live0 ? keys[i0] : 0u;
+      hist_add(hist, (key >> wlo) & (nbins - 1), live0 && (key & hmask) == (prefix & hmask));
+    }
+    cluster.sync();  // every slice histogram complete
+    // reduce-scatter + all-gather: this CTA sums bins [rank * nbins / 8, ...) over
+    // the 8 slices and writes the sums into every CTA's merged histogram
+    {
+      const int span = (int)nbins / kCluster > 0 ? (int)nbins / kCluster : 1;
+      const int b0 = rank * span;
+      for (int bin = b0 + tid; bin < min((int)nbins, b0 + span); bin += kCThreads) {
+        uint32_t v[kCluster];
+#pragma unroll
+        for (int r = 0; r < kCluster; ++r) v[r] = cluster.map_shared_rank(hist, r)[bin];  // independent loads
+        uint32_t sum = 0;
+#pragma unroll
+        for (int r = 0; r < kCluster; ++r) sum += v[r];
+#pragma unroll
+        for (int r = 0; r < kCluster; ++r) cluster.map_shared_rank(merged, r)[bin] = sum;
       }
-    } else {  // low bits: fetch the full key of the keys still matching the prefix
-      const uint32_t hm16 = hmask >> 16, hp16 = (prefix & hmask) >> 16;
-      for (int i0 = tid; i0 < ((n + 31) & ~31); i0 += kThreads) {
-        const bool live0 = i0 < n && ((uint32_t)hi16[min(i0, n - 1)] & hm16) == hp16;
-        const uint32_t key = live0 ? float_key(s[i0]) : 0u;
-        const bool live = live0 && (key & hmask) == (prefix & hmask);
-        hist_add(hist, (key >> lo) & (nbins - 1), live);
+      if ((int)nbins < kCluster) {  // tiny windows: rank 0 alone
+        if (rank == 0)
+          for (int bin = tid; bin < (int)nbins; bin += kCThreads) {
+            uint32_t sum = 0;
+            for (int r = 0; r < kCluster; ++r) sum += cluster.map_shared_rank(hist, r)[bin];
+            for (int r = 0; r < kCluster; ++r) cluster.map_shared_rank(merged, r)[bin] = sum;
+          }
       }
     }
-    __syncthreads();
-    find_bin(hist, (int)nbins, remaining, wsum, &s_bin, &s_above);
-    prefix |= (uint32_t)s_bin << lo;
-    remaining -= s_above;
-    hb = lo - 1;
+    cluster.sync();  // merged histogram complete everywhere; slice histograms free
+    uint32_t above;
+    const int b = cluster_find_bin(merged, (int)nbins, remaining, wsum, &s_bin, &s_above, &above);
+    prefix |= (uint32_t)b << wlo;
+    remaining -= above;
+    hb = wlo - 1;
   }
   const uint32_t T = prefix;          // the K-th largest key
   const uint32_t need_eq = remaining;  // keys equal to T to keep, lowest index first
-  const uint32_t T16 = T >> 16;
-  // ---- 3. bitmap of keys > T, per-word counts of keys == T
-  for (int w = warp; w < words; w += kWarps) {
+  // ---- ordered output.  Per 32-key word: counts of keys > T and == T (ballots)
+  const int words = (m + 31) >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int w = warp; w < words; w += kCWarps) {
     const int i = (w << 5) + lane;
-    const bool live = i < n;
-    const uint32_t h = live ? hi16[i] : 0u;
-    const bool tie16 = live && h == T16;
-    const uint32_t key = tie16 ? float_key(s[i]) : 0u;
-    const uint32_t gt = __ballot_sync(0xffffffffu, live && (h > T16 || (tie16 && key > T)));
-    const uint32_t eq = __ballot_sync(0xffffffffu, tie16 && key == T);
+    const uint32_t k = i < m ? keys[i] : 0u;
+    const uint32_t gt = __ballot_sync(0xffffffffu, i < m && k > T);
+    const uint32_t eq = __ballot_sync(0xffffffffu, i < m && k == T);
     if (lane == 0) {
-      bitmap[w] = gt;
-      wcnt[w] = __popc(eq);
+      wgt_cnt[w] = __popc(gt);
+      weq_cnt[w] = __popc(eq);
     }
   }
   __syncthreads();
-  block_exclusive_scan(wcnt, words, wsum);
-  for (int w = warp; w < words; w += kWarps) {
+  // slice totals, published for the higher-ranked CTAs
+  uint32_t g_loc = tid < words ? wgt_cnt[tid] : 0u, e_loc = tid < words ? weq_cnt[tid] : 0u;
+  uint32_t e_pre;
+  const uint32_t e_tot = block_exclusive(e_loc, wsum, &e_pre);
+  uint32_t g_pre;
+  const uint32_t g_tot = block_exclusive(g_loc, wsum, &g_pre);
+  if (tid == 0) {
+    pub[2] = g_tot;
+    pub[3] = e_tot;
+  }
+  cluster.sync();
+  uint32_t eq_before = 0, sel_before = 0;
+  for (int r = 0; r < rank; ++r) {
+    const uint32_t* rp = cluster.map_shared_rank(pub, r);
+    const uint32_t take_eq = need_eq > eq_before ? min(need_eq - eq_before, rp[3]) : 0u;
+    sel_before += rp[2] + take_eq;
+    eq_before += rp[3];
+  }
+  cluster.sync();  // remote reads of pub done before any CTA exits
+  // per word: ties before it (index order), keys it keeps, and its first output slot
+  uint32_t eqb = eq_before + e_pre;
+  const uint32_t take_w = tid < words ? (need_eq > eqb ? min(need_eq - eqb, e_loc) : 0u) + g_loc : 0u;
+  uint32_t sel_pre;
+  block_exclusive(take_w, wsum, &sel_pre);
+  if (tid < words) {
+    weq_cnt[tid] = eqb;                    // ties before this word
+    wgt_cnt[tid] = sel_before + sel_pre;   // first output slot of this word
+  }
+  __syncthreads();
+  for (int w = warp; w < words; w += kCWarps) {
     const int i = (w << 5) + lane;
-    const bool tie16 = i < n && hi16[i] == T16;
-    const bool e = tie16 && float_key(s[i]) == T;
-    const uint32_t eq = __ballot_sync(0xffffffffu, e);
-    const bool take = e && wcnt[w] + __popc(eq & lt) < need_eq;
+    const uint32_t k = i < m ? keys[i] : 0u;
+    const bool is_gt = i < m && k > T;
+    const bool is_eq = i < m && k == T;
+    const uint32_t eq = __ballot_sync(0xffffffffu, is_eq);
+    const bool take = is_gt || (is_eq && weq_cnt[w] + __popc(eq & lt) < need_eq);
     const uint32_t tk = __ballot_sync(0xffffffffu, take);
-    if (lane == 0 && tk) bitmap[w] |= tk;
+    if (take) out[wgt_cnt[w] + __popc(tk & lt)] = lo + i;
   }
-  __syncthreads();
-  // ---- 4. ascending emission from the bitmap: per-thread word runs + block scan
-  const int per = (words + kThreads - 1) / kThreads;
-  const int w0 = tid * per;
-  uint32_t cnt = 0;
-  for (int w = w0; w < min(words, w0 + per); ++w) cnt += __popc(bitmap[w]);
-  uint32_t inc = cnt;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const uint32_t v = __shfl_up_sync(0xffffffffu, inc, d);
-    if (lane >= d) inc += v;
-  }
-  if (lane == 31) wsum[warp] = inc;
-  __syncthreads();
-  uint32_t base = inc - cnt;
-  for (int w = 0; w < warp; ++w) base += wsum[w];
-  for (int w = w0; w < min(words, w0 + per); ++w) {
-    uint32_t bits = bitmap[w];
-    while (bits) {
-      const int b = __ffs(bits) - 1;
-      bits &= bits - 1;
-      out[base++] = w * 32 + b;
-    }
-  }
+}
+
+// Rows longer than the cluster path holds: one CTA per such query.
+__global__ void __launch_bounds__(kThreads) topk_long_kernel(TopkArgs a) {
+  __shared__ uint32_t hist[4096];
+  __shared__ uint32_t wsum[kWarps];
+  __shared__ uint32_t wgt[kWarps], weq[kWarps];
+  __shared__ int s_bin;
+  __shared__ uint32_t s_above;
+  const int q = blockIdx.x;
+  const int p = a.q_pos[q];
+  int64_t nb = p >= 0 ? (int64_t)(p + 1) / kRatio : 0;
+  if (nb > a.ld) nb = a.ld;
+  if (a.K == 0 || nb <= kMaxFast) return;  // handled by the cluster kernel
+  topk_general(a.scores + (size_t)q * a.ld, (int)nb, a.K, a.sel + (size_t)q * a.K, hist, wsum, wgt, weq, &s_bin,
+               &s_above);
 }
 
 }  // namespace
@@ -388,14 +451,15 @@ extern "C" int qsa_topk_blocks(const float* scores, int64_t scores_ld, const int
   if (nq < 0 || k < 0 || k > QSA_MAX_TOPK || scores_ld < 1) return QSA_ERR_INVALID_ARG;
   if (nq == 0) return QSA_OK;
   if (!scores || !q_pos || !count || (k > 0 && !sel)) return QSA_ERR_INVALID_ARG;
-  // shared-memory path sized for this call's rows: 2 B of key prefix + 8 B per 32 blocks
-  const int32_t fast_cap = (int32_t)((scores_ld < kMaxFast ? (scores_ld + 1023) / 1024 * 1024 : kMaxFast));
-  TopkArgs a{scores, scores_ld, q_pos, k, fast_cap, sel, count, dev_status};
-  const size_t smem = (size_t)fast_cap * 2 + (size_t)fast_cap / 32 * 4 * 2;
-  if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+  TopkArgs a{scores, scores_ld, q_pos, k, kMaxFast, sel, count, dev_status};
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSliceCap * 4) != cudaSuccess) {
     (void)cudaGetLastError();
     return QSA_ERR_CUDA;
   }
-  topk_kernel<<<(unsigned)nq, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(a);
+  topk_kernel<<<(unsigned)((int64_t)nq * kCluster), kCThreads, kSliceCap * 4, st>>>(a);
+  int rc = qsa_host::launch_status();
+  if (rc != QSA_OK) return rc;
+  if (scores_ld > kMaxFast) topk_long_kernel<<<(unsigned)nq, kThreads, 0, st>>>(a);
   return qsa_host::launch_status();
 }
