@@ -2,7 +2,7 @@
 
 The compute runs in libqsa.so (hand-written CUDA, C ABI in include/qsa.h); this
 package is its thin ctypes binding.  Build the library with
-``python -m sparse_attention_decode_03_b200.build``.
+``python sparse_attention_decode_03_b200/build.py``.
 """
 from .qsa import (  # noqa: F401
     ABI_VERSION, LIB_PATH, BoundCall, Decoder, bind_append_kv, PagedCache, QSAError, dev_status_names, qsa_append_kv, qsa_combine,

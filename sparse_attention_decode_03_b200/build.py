@@ -1,6 +1,6 @@
 """Build libqsa.so (the C-ABI CUDA library) in-tree for sm_100a.
 
-    python -m sparse_attention_decode_03_b200.build [--verbose]
+    python sparse_attention_decode_03_b200/build.py [--verbose]
 
 Compiles every csrc/*.cu with nvcc (-gencode arch=compute_100a,code=sm_100a)
 in parallel and links them into sparse_attention_decode_03_b200/libqsa.so.

@@ -47,7 +47,7 @@ class qsa_cache_t(ctypes.Structure):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libqsa.so not built at {LIB_PATH}; run `python -m sparse_attention_decode_03_b200.build`")
+        raise ImportError(f"libqsa.so not built at {LIB_PATH}; run `python sparse_attention_decode_03_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P, I32, I64, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
     PC = ctypes.POINTER(qsa_cache_t)
