@@ -218,6 +218,40 @@ QSA_API int qsa_sparse_decode(const qsa_cache_t* cache, const void* q, int32_t n
 QSA_API int qsa_combine(const float* part_o, const float* part_lse, int32_t nq, int32_t max_splits, int32_t hq,
                 void* out, float* lse, void* stream);
 
+/*
+ * qsa_sparse_attention_noalloc -- qsa_sparse_decode then qsa_combine in one
+ * call, for callers that cannot allocate device memory.  The pages have no
+ * counterpart to this call; it is a convenience of this library.
+ *
+ * Some callers cannot call cudaMalloc: a serving engine that hands nearly all
+ * device memory to its KV-cache pool at start-up, a plug-in whose host program
+ * owns every device allocation, or a latency-critical loop that must not take
+ * cudaMalloc's implicit device synchronisation.  This call needs no buffer
+ * beyond its inputs and outputs: it keeps the split partials in a device array
+ * of QSA_NOALLOC_SCRATCH_BYTES that libqsa reserves itself.  This is the one
+ * exception to "the library allocates nothing": every GPU that loads the
+ * library holds that array until the process exits.
+ *
+ * Arguments: as qsa_sparse_decode, with max_splits = the split bound that
+ * qsa_decode_plan reports for (k, chunk_units); out and lse as qsa_combine
+ * (bf16 [nq][hq][256] and fp32 [nq][hq]; out 8-byte aligned).
+ * Limit: nq * S * hq * 1028 bytes of partials (S = that split bound) must fit
+ * in QSA_NOALLOC_SCRATCH_BYTES; a larger call returns QSA_ERR_UNSUPPORTED and
+ * enqueues nothing.
+ * First call per device: it looks up the array's device address with that
+ * device current and caches it.  Make the first call on each device before
+ * any stream capture.
+ * Sharing: all calls on a device use the same array, which keeps the last
+ * call's contents (every partial the combine reads is rewritten by each call,
+ * so nothing needs clearing).  Calls whose kernels can overlap on the GPU
+ * (unordered streams, several host threads) race on the array: order them.
+ */
+#define QSA_NOALLOC_SCRATCH_BYTES (16u << 20)
+QSA_API int qsa_sparse_attention_noalloc(const qsa_cache_t* cache, const void* q, int32_t nq, int32_t hq,
+                                 const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel,
+                                 const int32_t* count, int32_t k, float scale, int32_t chunk_units, void* out,
+                                 float* lse, int32_t* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -60,6 +60,7 @@ def _load() -> ctypes.CDLL:
         "qsa_decode_plan": (ctypes.c_int, [I32, I32, I32, I32, ctypes.POINTER(I32), ctypes.POINTER(I32)]),
         "qsa_sparse_decode": (ctypes.c_int, [PC, P, I32, I32, P, P, P, P, I32, F, I32, I32, P, P, P, P]),
         "qsa_combine": (ctypes.c_int, [P, P, I32, I32, I32, P, P, P]),
+        "qsa_sparse_attention_noalloc": (ctypes.c_int, [PC, P, I32, I32, P, P, P, P, I32, F, I32, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -229,6 +230,33 @@ def qsa_combine(part_o, part_lse, out, lse, stream=None):
     _req(lse, "lse", torch.float32, (nq, hq))
     _check("qsa_combine", LIB.qsa_combine(_ptr(part_o), _ptr(part_lse), nq, S, hq, _ptr(out), _ptr(lse),
                                           _stream(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def qsa_sparse_attention_noalloc(cache: PagedCache, q, q_seq, q_pos, sel, count, k: int, scale: float,
+                                 chunk_units: int, out, lse, dev_status=None, stream=None):
+    """qsa_sparse_decode + qsa_combine for callers that cannot allocate device
+    memory: the split partials live in a fixed device array of
+    NOALLOC_SCRATCH_BYTES inside libqsa.  Calls on one device share that array,
+    so calls that can overlap on the GPU must be ordered (one stream).  The
+    first call on each device looks up the array's address; make it before any
+    stream capture."""
+    nq = int(q_seq.shape[0])
+    hq = int(q.shape[1]) if q.dim() == 3 else -1
+    _req(q, "q", torch.bfloat16, (nq, hq, HEAD_DIM))
+    _req(q_seq, "q_seq", torch.int32, (nq,))
+    _req(q_pos, "q_pos", torch.int32, (nq,))
+    _req(sel, "sel", torch.int32, (nq, k))
+    _req(count, "count", torch.int32, (nq,))
+    _req(out, "out", torch.bfloat16, (nq, hq, HEAD_DIM))
+    _req(lse, "lse", torch.float32, (nq, hq))
+    if dev_status is not None:
+        _req(dev_status, "dev_status", torch.int32, (1,))
+    _check("qsa_sparse_attention_noalloc", LIB.qsa_sparse_attention_noalloc(
+        ctypes.byref(cache.struct()), _ptr(q), nq, hq, _ptr(q_seq), _ptr(q_pos), _ptr(sel), _ptr(count), int(k),
+        float(scale), int(chunk_units), _ptr(out), _ptr(lse), _ptr(dev_status), _stream(stream)))
 
 
 # ----------------------------------------------------------------------------
