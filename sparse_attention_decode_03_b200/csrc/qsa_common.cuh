@@ -135,6 +135,20 @@ QSA_DEVINL void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t
       : "memory");
 }
 
+// 16-byte async copy global -> shared (L2 only, cache hint); 16-byte aligned.
+QSA_DEVINL void cp_async16(uint32_t dst, const void* src, uint64_t policy) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "l"(policy)
+               : "memory");
+}
+
+// Arrive on `bar` once every cp.async this thread issued so far has landed; the
+// arrival counts toward the barrier's expected count (noinc).
+QSA_DEVINL void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+QSA_DEVINL void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // Fire-and-forget prefetch of [src, src+bytes) into L2 (16-byte aligned, multiple of 16).
 QSA_DEVINL void prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");

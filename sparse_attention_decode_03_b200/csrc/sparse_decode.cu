@@ -16,15 +16,17 @@
 // same number of slots whatever the batch shape.  The part of a pair inside a
 // chunk is a "segment"; each segment yields one split partial.
 //
-// CTA = 4 consumer warps + a copy warp + a lookup warp, 1 CTA per SM.
+// CTA = 8 consumer warps + 2 copy warps + a lookup warp, 1 CTA per SM.
 //   lookup warp: walks the CTA's units 32 at a time (selection -> page table)
 //     and writes their source offsets into a 3-batch descriptor queue, so the
 //     dependent selection and page-table loads run ahead of the copies.
-//   copy warp: per tile of 4 units issues one cp.async.bulk copy of 4 KiB per
-//     unit into an 8-stage shared-memory ring (mbarrier full/empty pairs).
-//     The bulk-copy engine costs about a hundred cycles per operation on B200,
-//     whatever its size; 4 KiB operations keep it near HBM speed where 2 KiB
-//     ones cap an SM at about two thirds of its share.
+//   copy warps: tile T (4 units) belongs to copy warp T % 2, which moves each
+//     unit's 4 KiB with 16-byte cp.async copies (every lane 8 per unit) into
+//     an 8-stage shared-memory ring; each lane then arrives on the stage's
+//     mbarrier when its copies land (cp.async.mbarrier.arrive.noinc).  With
+//     one issuing thread per SM (a 1-D bulk copy per unit) random 4 KiB
+//     gathers stayed near half the HBM rate on B200; spreading the issue over
+//     the lanes of more warps is what raises the gather rate.
 //   consumers: 4 pairs of warps; tile T (16 tokens) belongs to pair T % 4.
 //     Both warps of a pair compute S = Q K^T for the tile and the online
 //     softmax (mma.sync m16n8k16, M = 16 Q-head rows of the KV group, fp32
@@ -42,9 +44,10 @@ using namespace qsa;
 
 constexpr int kConsumerWarps = 8;                 // 4 pairs
 constexpr int kPairs = kConsumerWarps / 2;
-constexpr int kCopyWarp = kConsumerWarps;         // warp 8
-constexpr int kLookupWarp = kConsumerWarps + 1;   // warp 9
-constexpr int kThreads = (kConsumerWarps + 2) * 32;
+constexpr int kCopyWarps = 2;
+constexpr int kCopyWarp0 = kConsumerWarps;                // warps 8, 9
+constexpr int kLookupWarp = kConsumerWarps + kCopyWarps;  // warp 10
+constexpr int kThreads = (kLookupWarp + 1) * 32;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 // A stage is reused by tile T + kStages; with kStages a multiple of the consumer
 // pair count and tile T owned by pair T % 4, that tile's owner is the pair that
@@ -53,7 +56,8 @@ constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kStages = 8;
 constexpr int kUnitsPerTile = 4;
 constexpr int kBatch = 32;                                             // units per lookup batch
-constexpr int kDescSlots = 3;                                          // lookup batches in flight
+constexpr int kRound = 4;                                              // lookup batches resolved together
+constexpr int kDescSlots = 2 * kRound;                                 // lookup batches in flight
 constexpr int kHalfBytes = kRatio * kHeadDim * 2;                      // 2048: 4 K (or V) rows
 constexpr int kUnitBytes = 2 * kHalfBytes;                             // 4096: K rows then V rows
 constexpr int kSlotStride = kUnitBytes + 32;                           // 4128: 16-B bank-group skew of 2
@@ -74,7 +78,10 @@ constexpr int kNumBars = 2 * kStages + 2 * kDescSlots;
 constexpr int kOffAbort = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffAbort + 16;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kStages % kPairs == 0, "tile ownership must repeat with the stage ring");
+static_assert(kStages % kPairs == 0 && kStages % kCopyWarps == 0, "tile ownership must repeat with the stage ring");
+// full barrier: the 32 lanes' copy-completion arrivals + the owning copy warp's
+// lane 0, whose plain (release) arrival publishes the stage's row mask
+constexpr int kFullArrivals = 33;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr int kBarConsumers = 1;                  // named barrier id
 constexpr uint64_t kNoCopy = ~0ull;
@@ -215,6 +222,9 @@ __device__ __forceinline__ bool warp_aborted(volatile int* abort_flag) {
   return __shfl_sync(0xffffffffu, v, 0) != 0;
 }
 
+// Resolves kRound batches per round: the selection loads of all of them are
+// issued together, then the page-table loads, so a round costs two dependent
+// global-load latencies for 4 x 32 units.
 __device__ void lookup_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_t x1) {
   const int lane = threadIdx.x & 31;
   uint64_t* d_off = reinterpret_cast<uint64_t*>(smem + kOffDescOff);
@@ -224,48 +234,84 @@ __device__ void lookup_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int6
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
   BatchIter it;
   bool have = iter_begin(a, it, x0, x1);
-  for (int b = 0; have; ++b, have = iter_next(a, it)) {
-    const int slot = b % kDescSlots;
-    if (b >= kDescSlots && !warp_wait(a, bar_dempty + slot * 8, (uint32_t)((b / kDescSlots - 1) & 1), abort_flag))
-      return;
-    if (warp_aborted(abort_flag)) return;
-    const Seg& s = it.s;
-    const int i = it.ub + lane;
-    uint32_t rows = 0;
-    uint64_t off = kNoCopy;
-    if (i < s.n_valid) {
-      int j, nrows;
-      bool ok = true;
-      if (i < s.n_main) {
-        j = a.sel[(size_t)s.q * a.K + s.u0 + i];
-        nrows = kRatio;
-        if (j < 0 || j >= s.nb) {
-          flag(a.st, QSA_DEV_BAD_SEL);
-          ok = false;
-        }
-      } else {
-        j = s.nb;
-        nrows = s.t;
+  int b = 0;
+  while (have) {
+    int nr = 0;
+    int q[kRound], seq[kRound], nb[kRound], t[kRound], sel_base[kRound], g[kRound], i_main[kRound], i_valid[kRound];
+#pragma unroll
+    for (int r = 0; r < kRound; ++r) {
+      if (have) {  // warp-uniform
+        const Seg& sg = it.s;
+        q[r] = sg.q;
+        g[r] = sg.g;
+        seq[r] = sg.seq;
+        nb[r] = sg.nb;
+        t[r] = sg.t;
+        sel_base[r] = sg.u0 + it.ub;
+        i_main[r] = sg.n_main - it.ub;   // this batch's units below i_main are selected blocks
+        i_valid[r] = sg.n_valid - it.ub; // ... below i_valid are valid (the tail last)
+        nr = r + 1;
+        have = iter_next(a, it);
       }
-      if (ok) {
-        const int phys = a.bt[(int64_t)s.seq * a.mpps + j / kBlocksPerPage];
-        if (phys < 0 || phys >= a.num_pages) {
-          flag(a.st, QSA_DEV_BAD_PAGE);
+    }
+    // 1. selection entries of every batch in the round (independent loads)
+    int j[kRound];
+    bool ok[kRound];
+#pragma unroll
+    for (int r = 0; r < kRound; ++r) {
+      ok[r] = false;
+      j[r] = 0;
+      if (r < nr && lane < i_valid[r]) {
+        if (lane < i_main[r]) {
+          j[r] = a.sel[(size_t)q[r] * a.K + sel_base[r] + lane];
+          ok[r] = true;
         } else {
-          off = (((uint64_t)phys * a.hkv + s.g) * kBlocksPerPage + (uint64_t)(j % kBlocksPerPage)) *
-                (2 * kRatio * kHeadDim);
-          rows = (1u << nrows) - 1u;
+          j[r] = nb[r];
+          ok[r] = true;
         }
       }
     }
-    d_off[slot * kBatch + lane] = off;
-    d_rows[slot * kBatch + lane] = rows;
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar_dfull + slot * 8);
+#pragma unroll
+    for (int r = 0; r < kRound; ++r) {
+      if (ok[r] && lane < i_main[r] && (j[r] < 0 || j[r] >= nb[r])) {
+        flag(a.st, QSA_DEV_BAD_SEL);
+        ok[r] = false;
+      }
+    }
+    // 2. page-table entries (independent loads)
+    int phys[kRound];
+#pragma unroll
+    for (int r = 0; r < kRound; ++r) phys[r] = ok[r] ? a.bt[(int64_t)seq[r] * a.mpps + j[r] / kBlocksPerPage] : -1;
+    // 3. publish each batch's descriptors once its queue slot is free
+#pragma unroll
+    for (int r = 0; r < kRound; ++r) {
+      if (r >= nr) break;
+      const int bb = b + r;
+      const int slot = bb % kDescSlots;
+      if (bb >= kDescSlots && !warp_wait(a, bar_dempty + slot * 8, (uint32_t)((bb / kDescSlots - 1) & 1), abort_flag))
+        return;
+      if (warp_aborted(abort_flag)) return;
+      uint64_t off = kNoCopy;
+      uint32_t rows = 0;
+      if (ok[r]) {
+        if (phys[r] < 0 || phys[r] >= a.num_pages) {
+          flag(a.st, QSA_DEV_BAD_PAGE);
+        } else {
+          off = (((uint64_t)phys[r] * a.hkv + g[r]) * kBlocksPerPage + (uint64_t)(j[r] % kBlocksPerPage)) *
+                (2 * kRatio * kHeadDim);
+          rows = lane < i_main[r] ? 0xFu : (1u << t[r]) - 1u;
+        }
+      }
+      d_off[slot * kBatch + lane] = off;
+      d_rows[slot * kBatch + lane] = rows;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_dfull + slot * 8);
+    }
+    b += nr;
   }
 }
 
-__device__ void copy_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_t x1) {
+__device__ void copy_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_t x1, int cw) {
   const int lane = threadIdx.x & 31;
   const uint32_t ring = smem_u32(smem + kOffRing);
   const uint32_t bar_full = smem_u32(smem + kOffBar);
@@ -277,6 +323,7 @@ __device__ void copy_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
   uint32_t* meta = reinterpret_cast<uint32_t*>(smem + kOffMeta);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
   const uint64_t policy = l2_policy_evict_first();
+  const char* kv = reinterpret_cast<const char*>(a.kv_pages);
   int64_t T = 0;
   BatchIter it;
   bool have = iter_begin(a, it, x0, x1);
@@ -286,11 +333,12 @@ __device__ void copy_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
     const uint64_t off = d_off[slot * kBatch + lane];
     const uint32_t rows = d_rows[slot * kBatch + lane];
     __syncwarp();
-    if (lane == 0) mbar_arrive(bar_dempty + slot * 8);
+    if (lane == 0) mbar_arrive(bar_dempty + slot * 8);  // both copy warps arrive
     const int n_units = min(kBatch, it.s.n_valid - it.ub);
     const int tiles = (n_units + kUnitsPerTile - 1) / kUnitsPerTile;
     bool stop = false;
     for (int tb = 0; tb < tiles; ++tb, ++T) {
+      if ((int)(T % kCopyWarps) != cw) continue;
       const int stage = (int)(T % kStages);
       if (T >= kStages && !warp_wait(a, bar_empty + stage * 8, (uint32_t)((T / kStages - 1) & 1), abort_flag)) {
         stop = true;
@@ -301,26 +349,27 @@ __device__ void copy_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
         break;
       }
       const bool mine = (lane >> 2) == tb && lane < n_units;
-      const int slot4 = lane & 3;
-      const bool do_copy = mine && off != kNoCopy;
-      const uint32_t rowmask = __reduce_or_sync(0xffffffffu, mine ? (rows << (slot4 * 4)) : 0u);
-      const uint32_t ncopy = __popc(__ballot_sync(0xffffffffu, do_copy));
+      const uint32_t rowmask = __reduce_or_sync(0xffffffffu, mine ? (rows << ((lane & 3) * 4)) : 0u);
+      const uint32_t dst = ring + stage * kStageBytes + lane * 16;
+#pragma unroll
+      for (int u = 0; u < kUnitsPerTile; ++u) {
+        const uint64_t uoff = __shfl_sync(0xffffffffu, off, (tb * kUnitsPerTile + u) & 31);
+        if (tb * kUnitsPerTile + u < n_units && uoff != kNoCopy) {
+          const char* src = kv + uoff * sizeof(__nv_bfloat16) + lane * 16;
+#pragma unroll
+          for (int c = 0; c < kUnitBytes / 512; ++c) cp_async16(dst + u * kSlotStride + c * 512, src + c * 512, policy);
+        }
+      }
       if (lane == 0) {
         meta[stage] = rowmask;
-        mbar_arrive_expect_tx(bar_full + stage * 8, ncopy * kUnitBytes);
+        mbar_arrive(bar_full + stage * 8);
       }
-      __syncwarp();
-      if (do_copy)
-        bulk_g2s(ring + stage * kStageBytes + slot4 * kSlotStride, a.kv_pages + off, kUnitBytes,
-                 bar_full + stage * 8, policy);
+      cp_async_arrive_noinc(bar_full + stage * 8);
     }
     if (stop) break;
   }
-  // Never leave the CTA with copies in flight: wait for the last tiles' data.
-  if (lane == 0) {
-    for (int64_t k = T > kStages ? T - kStages : 0; k < T; ++k)
-      mbar_wait_bounded(bar_full + (int)(k % kStages) * 8, (uint32_t)((k / kStages) & 1), kWaitLimitNs);
-  }
+  // Never leave the CTA with copies in flight.
+  cp_async_wait_all();
   __syncwarp();
 }
 
@@ -619,12 +668,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(DecodeArgs a
   if (threadIdx.x == 0) {
     const uint32_t bf = smem_u32(smem + kOffBar);
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(bf + i * 8, 1);                  // full: copy warp's arrive + tx bytes
+      mbar_init(bf + i * 8, kFullArrivals);      // full: copy completions + row mask published
       mbar_init(bf + (kStages + i) * 8, 2);      // empty: both warps of the owning pair
     }
     for (int i = 0; i < kDescSlots; ++i) {
       mbar_init(bf + (2 * kStages + i) * 8, 1);               // descriptors written (lookup warp)
-      mbar_init(bf + (2 * kStages + kDescSlots + i) * 8, 1);  // descriptors taken (copy warp)
+      mbar_init(bf + (2 * kStages + kDescSlots + i) * 8, kCopyWarps);  // descriptors taken (copy warps)
     }
     *reinterpret_cast<volatile int*>(smem + kOffAbort) = 0;
     fence_mbar_init();
@@ -632,8 +681,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(DecodeArgs a
   __syncthreads();
   if (x0 >= x1) return;
   const int warp = threadIdx.x >> 5;
-  if (warp == kCopyWarp)
-    copy_warp(a, smem, x0, x1);
+  if (warp >= kCopyWarp0 && warp < kCopyWarp0 + kCopyWarps)
+    copy_warp(a, smem, x0, x1, warp - kCopyWarp0);
   else if (warp == kLookupWarp)
     lookup_warp(a, smem, x0, x1);
   else

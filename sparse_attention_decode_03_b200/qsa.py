@@ -366,6 +366,43 @@ class Decoder:
         return self.out[:nq], self.lse[:nq]
 
 
+class StepGraph:
+    """The pre-bound launches of one step captured once into a CUDA graph and
+    replayed with a single launch, so a step costs no per-kernel host work.
+    The library calls only enqueue kernels (no allocation, no host
+    synchronisation), which is what lets them be captured.  The calls must have
+    been bound to `stream` (a side stream, not the legacy default stream).
+
+    With ``timing=True`` a timing event is captured before every call and
+    after the last one; after a replay, :meth:`kernel_ms` gives each call's
+    device time for that replay."""
+
+    def __init__(self, calls, stream: torch.cuda.Stream, timing: bool = False):
+        self.calls = list(calls)
+        self.stream = stream
+        self.events = ([torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(self.calls) + 1)]
+                       if timing else None)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=stream):
+            for k, c in enumerate(self.calls):
+                if self.events:
+                    self.events[k].record(stream)
+                c()
+            if self.events:
+                self.events[-1].record(stream)
+
+    def replay(self):
+        """Enqueue one replay on the graph's stream (stream-ordered after the
+        work already enqueued there)."""
+        with torch.cuda.stream(self.stream):
+            self.graph.replay()
+
+    def kernel_ms(self) -> list:
+        """Device time of each call in the last replay (synchronises on it)."""
+        self.events[-1].synchronize()
+        return [self.events[k].elapsed_time(self.events[k + 1]) for k in range(len(self.calls))]
+
+
 def splits_bound(k: int, chunk_units: int) -> int:
     """Most KV chunks one (query, KV head) pair's k+1 unit slots can touch."""
     return (k + 1 + chunk_units - 2) // chunk_units + 1
