@@ -6,28 +6,27 @@
 // the tie-break (lower index first) and ascending output order are the fixed
 // readings.
 //
-// Order-preserving uint32 keys of the fp32 scores.  One thread-block cluster
-// of 8 CTAs per query (decode batches have only 32-64 queries, so a single CTA
-// per query leaves the per-key work on too few SMs).  CTA r of the cluster owns
-// the r-th contiguous eighth of the row and keeps its keys in shared memory
-// after one vectorised read.  Then:
-//   1. cluster-wide min / max key (distributed shared memory);
-//   2. radix select with adaptive 11-bit windows starting at the highest bit
-//      where the keys differ (scores share their top exponent bits): every CTA
-//      histograms its slice, the 8 histograms are summed through distributed
-//      shared memory, and each CTA finds the same bin; this yields the exact
-//      K-th largest key T;
-//   3. each CTA ranks its keys == T in index order (word ballots, a block scan
-//      and the counts of the lower-ranked CTAs) and keeps the lowest-index
-//      ones, then writes its selected indices, in ascending order, at the
-//      offset given by the lower-ranked CTAs' counts.
-// Rows longer than 65,536 blocks take the general path in the cluster's first
-// CTA: three radix passes over the scores (12 + 12 + 8 bits) and an ordered
-// compaction with warp ballots.
-// Integer counters only: the result does not depend on atomic order.
+// Order-preserving uint32 keys of the fp32 scores; one CTA of 1024 threads per
+// query.  A histogram pass over a whole row costs about one cycle per key of
+// one SM's shared-memory atomics, so only small sets are histogrammed:
+//   1. threshold: 1024 keys sampled at a regular stride are histogrammed (12-bit
+//      window from their highest differing bit); T0 is the lower edge of the
+//      bin where the count from the top reaches r = K*1024/n plus a margin of
+//      three standard deviations, so that about r*n/1024 >= K keys are >= T0;
+//   2. candidates: each warp streams its contiguous 1/32 of the row (16-byte
+//      loads) and appends the keys >= T0 with their indices to its own
+//      shared-memory list, in index order (ballots and a warp scan);
+//   3. exact select among the candidates: radix passes (12-bit windows from
+//      the candidates' highest differing bit, warp-aggregated atomics) give a
+//      prefix T under a mask with "every key above T, and the first `need`
+//      keys equal to T in index order" = the top K;
+//   4. ordered output: warp totals scanned once, then each warp writes its
+//      kept indices in order.
+// If the sample misleads (fewer than K candidates, or more than a warp's list
+// holds) the CTA instead runs the general exact path: three radix passes over
+// the row in global memory and an ordered compaction.  Integer counters only:
+// the result does not depend on atomic order.
 #include "qsa_common.cuh"
-
-#include <cooperative_groups.h>
 
 namespace {
 
@@ -82,14 +81,7 @@ __device__ void find_bin(const uint32_t* hist, int nbins, uint32_t remaining, ui
   __syncthreads();
 }
 
-constexpr int kCluster = 8;                    // CTAs per query
-constexpr int kCThreads = 512;                 // threads per cluster CTA
-constexpr int kCWarps = kCThreads / 32;
-constexpr int kSliceCap = 8192;                // keys per CTA on the cluster path
-constexpr int kMaxFast = kCluster * kSliceCap; // 65,536 blocks per query
 constexpr int kUnroll = 8;
-constexpr int kWin = 11;                       // radix window bits
-constexpr int kWinBins = 1 << kWin;
 
 __device__ __forceinline__ void load_keys(const float* s, int i0, int n, uint32_t (&key)[kUnroll]) {
 #pragma unroll
@@ -166,282 +158,307 @@ __device__ void topk_general(const float* s, int n, int K, int32_t* out, uint32_
   }
 }
 
-// Shared-memory histogram increment.  A warp whose live lanes all hit one bin
-// (common when scores crowd together) adds once; otherwise per-lane atomics.
+constexpr int kSample = 1024;   // keys sampled for the threshold (one per thread)
+constexpr int kCap = 256;       // candidates one warp's list holds
+constexpr int kWin = 12;        // radix window bits
+constexpr int kWinBins = 1 << kWin;
+
+struct TopkSmem {
+  uint32_t ckey[kWarps][kCap];  // candidate keys, per warp, in index order
+  uint32_t cidx[kWarps][kCap];  // their block indices
+  uint32_t hist[kWinBins];
+  uint32_t wcnt[kWarps];        // candidates per warp (kCap + 1: overflow)
+  uint32_t wgt[kWarps], weq[kWarps], wslot[kWarps], weqb[kWarps];
+  uint32_t wsum[kWarps];
+  uint32_t red[2 * kWarps];
+  int bin;
+  uint32_t above;
+};
+
+// Add 1 to hist[bin] for every live lane: one atomic per distinct bin per warp.
 __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool live) {
   const uint32_t act = __ballot_sync(0xffffffffu, live);
-  if (act == 0) return;
-  const int leader = __ffs(act) - 1;
-  const uint32_t b0 = __shfl_sync(0xffffffffu, bin, leader);
-  if (__all_sync(0xffffffffu, !live || bin == b0)) {
-    if ((threadIdx.x & 31) == leader) atomicAdd(&hist[b0], (uint32_t)__popc(act));
-  } else if (live) {
-    atomicAdd(&hist[bin], 1u);
+  if (live) {
+    const uint32_t peers = __match_any_sync(act, bin);
+    if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
   }
 }
 
-// Bin b of a merged histogram (every thread returns the same) with
-// sum_{i > b} hist[i] < remaining <= sum_{i >= b} hist[i]; *above = sum_{i > b}.
-__device__ int cluster_find_bin(const uint32_t* hist, int nbins, uint32_t remaining, uint32_t* wsum, int* s_bin,
-                                uint32_t* s_above, uint32_t* above) {
+// Block-wide min and max of one value per thread.
+__device__ __forceinline__ void block_minmax(uint32_t& mn, uint32_t& mx, uint32_t* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  mn = __reduce_min_sync(0xffffffffu, mn);
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  if (lane == 0) {
+    red[warp] = mn;
+    red[kWarps + warp] = mx;
+  }
+  __syncthreads();
+  mn = __reduce_min_sync(0xffffffffu, red[lane]);
+  mx = __reduce_max_sync(0xffffffffu, red[kWarps + lane]);
+  __syncthreads();
+}
+
+// The bin b of hist[0..nbins) (counting from the top) with
+// sum_{>b} < remaining <= sum_{>=b}; *above = sum_{>b}.  Same result in every thread.
+__device__ int top_bin(const uint32_t* hist, int nbins, uint32_t remaining, TopkSmem& S, uint32_t* above) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int per = (nbins + kCThreads - 1) / kCThreads;
-  const int lo = tid * per;
+  const int per = (nbins + kThreads - 1) / kThreads;
+  const int b0 = tid * per;
   uint32_t local = 0;
-  for (int i = 0; i < per; ++i)
-    if (lo + i < nbins) local += hist[lo + i];
+  for (int j = 0; j < per; ++j)
+    if (b0 + j < nbins) local += hist[b0 + j];
   uint32_t suf = local;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
     const uint32_t v = __shfl_down_sync(0xffffffffu, suf, d);
     if (lane + d < 32) suf += v;
   }
-  if (lane == 0) wsum[warp] = suf;
+  if (lane == 0) S.wsum[warp] = suf;
   __syncthreads();
-  uint32_t cum = suf - local;
-  for (int w = warp + 1; w < kCWarps; ++w) cum += wsum[w];
-  for (int i = per - 1; i >= 0; --i) {
-    if (lo + i >= nbins) continue;
-    const uint32_t h = hist[lo + i];
+  // sum of the totals of the warps above mine: a suffix scan across lanes
+  const uint32_t wt = S.wsum[lane];
+  uint32_t wsuf = wt;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const uint32_t v = __shfl_down_sync(0xffffffffu, wsuf, d);
+    if (lane + d < 32) wsuf += v;
+  }
+  uint32_t cum = suf - local + (__shfl_sync(0xffffffffu, wsuf, warp) - __shfl_sync(0xffffffffu, wt, warp));
+  for (int j = per - 1; j >= 0; --j) {
+    if (b0 + j >= nbins) continue;
+    const uint32_t h = hist[b0 + j];
     if (cum < remaining && remaining <= cum + h) {
-      *s_bin = lo + i;
-      *s_above = cum;
+      S.bin = b0 + j;
+      S.above = cum;
     }
     cum += h;
   }
   __syncthreads();
-  *above = *s_above;
-  return *s_bin;
+  const int b = S.bin;
+  *above = S.above;
+  __syncthreads();  // S.bin / S.above / hist read everywhere before reuse
+  return b;
 }
 
-// Block-wide exclusive prefix of one value per thread; returns the block total.
-__device__ uint32_t block_exclusive(uint32_t v, uint32_t* wsum, uint32_t* prefix) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t inc = v;
+constexpr int kBatch = 8;  // 128-key chunks a warp loads at once
+
+// Load the chunks c0 + u*128 (u < kBatch) of [., hi): lane holds keys 4*lane .. 4*lane+3 of each.
+__device__ __forceinline__ void load_batch(const float* s, int c0, int hi, bool vec, float4 (&v)[kBatch]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int u = 0; u < kBatch; ++u) {
+    const int i0 = c0 + u * 128 + 4 * lane;
+    if (vec && i0 + 3 < hi) {
+      v[u] = __ldg(reinterpret_cast<const float4*>(s + i0));
+    } else {
+      v[u].x = i0 + 0 < hi ? __ldg(s + i0 + 0) : 0.f;
+      v[u].y = i0 + 1 < hi ? __ldg(s + i0 + 1) : 0.f;
+      v[u].z = i0 + 2 < hi ? __ldg(s + i0 + 2) : 0.f;
+      v[u].w = i0 + 3 < hi ? __ldg(s + i0 + 3) : 0.f;
+    }
+  }
+}
+
+// Append lane's flagged keys (f0..f3 of idx0..idx0+3) to this warp's list, in index order.
+__device__ __forceinline__ void append4(TopkSmem& S, int warp, uint32_t& cnt, const uint32_t (&k)[4], int idx0,
+                                        const bool (&f)[4]) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t nc = (uint32_t)f[0] + f[1] + f[2] + f[3];
+  uint32_t inc = nc;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
     const uint32_t x = __shfl_up_sync(0xffffffffu, inc, d);
     if (lane >= d) inc += x;
   }
-  if (lane == 31) wsum[warp] = inc;
-  __syncthreads();
-  uint32_t base = inc - v, total = 0;
-  for (int w = 0; w < kCWarps; ++w) {
-    if (w < warp) base += wsum[w];
-    total += wsum[w];
-  }
-  __syncthreads();
-  *prefix = base;
-  return total;
+  const uint32_t tot = __shfl_sync(0xffffffffu, inc, 31);
+  uint32_t pos = cnt + inc - nc;
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    if (f[c]) {
+      if (pos < kCap) {
+        S.ckey[warp][pos] = k[c];
+        S.cidx[warp][pos] = (uint32_t)(idx0 + c);
+      }
+      ++pos;
+    }
+  cnt += tot;
 }
 
-__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kCThreads) topk_kernel(TopkArgs a) {
-  namespace cg = cooperative_groups;
-  cg::cluster_group cluster = cg::this_cluster();
-  extern __shared__ __align__(16) uint32_t keys[];  // [kSliceCap] this CTA's slice of keys (dynamic)
-  __shared__ uint32_t hist[kWinBins];    // this slice's histogram
-  __shared__ uint32_t merged[kWinBins];  // the cluster's histogram (written by all 8 CTAs)
-  __shared__ uint32_t wgt_cnt[kSliceCap / 32], weq_cnt[kSliceCap / 32];
-  __shared__ uint32_t wsum[kCWarps];
-  __shared__ uint32_t pub[4];  // published per CTA: min key, max key, #keys > T, #keys == T
-  __shared__ int s_bin;
-  __shared__ uint32_t s_above;
-
-  const int rank = (int)cluster.block_rank();
-  const int q = blockIdx.x / kCluster;
+__global__ void __launch_bounds__(kThreads, 1) topk_kernel(TopkArgs a) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  TopkSmem& S = *reinterpret_cast<TopkSmem*>(smem_raw);
+  const int q = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int p = a.q_pos[q];
   int64_t nb = p >= 0 ? (int64_t)(p + 1) / kRatio : 0;
-  if (rank == 0 && tid == 0 && p < 0) flag(a.st, QSA_DEV_BAD_POS);
+  if (tid == 0 && p < 0) flag(a.st, QSA_DEV_BAD_POS);
   if (nb > a.ld) {
-    if (rank == 0 && tid == 0) flag(a.st, QSA_DEV_SCORES_LD);
+    if (tid == 0) flag(a.st, QSA_DEV_SCORES_LD);
     nb = a.ld;
   }
   const int K = a.K;
   int32_t* out = a.sel + (size_t)q * K;
-  // uniform early exits (every CTA of the cluster takes the same branch, before any cluster barrier)
   if (K == 0) {
-    if (rank == 0 && tid == 0) a.count[q] = 0;
+    if (tid == 0) a.count[q] = 0;
     return;
   }
   if (nb <= K) {  // every visible block is kept
-    if (rank == 0) {
-      for (int i = tid; i < K; i += kCThreads) out[i] = i < nb ? i : -1;
-      if (tid == 0) a.count[q] = (int32_t)nb;
-    }
+    for (int i = tid; i < K; i += kThreads) out[i] = i < nb ? i : -1;
+    if (tid == 0) a.count[q] = (int32_t)nb;
     return;
   }
-  const int n = (int)nb;
+  if (tid == 0) a.count[q] = K;
+  const int n = (int)min(nb, (int64_t)0x7fffffff);
   const float* s = a.scores + (size_t)q * a.ld;
-  if (n > kMaxFast) {  // selection written by topk_long_kernel, launched after this one
-    if (rank == 0 && tid == 0) a.count[q] = K;
+
+  // Each warp owns a contiguous segment of the row (a multiple of 128 keys).
+  // Its first kBatch x 128 keys are loaded now, so that their latency hides
+  // behind the threshold phase.
+  const int seg = (int)(((int64_t)n + 32 * 128 - 1) / (32 * 128)) * 128;
+  const int w_lo = min(n, warp * seg), w_hi = min(n, w_lo + seg);
+  const bool vec = (reinterpret_cast<uintptr_t>(s) & 15u) == 0;
+  float4 v[kBatch];
+  load_batch(s, w_lo, w_hi, vec, v);
+
+  // ---- 1. threshold T0 from a regular sample
+  const int ns = min(n, kSample);
+  const bool live_s = tid < ns;
+  const uint32_t ks = live_s ? float_key(__ldg(s + (int64_t)tid * n / ns)) : 0u;
+  uint32_t smin = live_s ? ks : 0xffffffffu, smax = live_s ? ks : 0u;
+  block_minmax(smin, smax, S.red);
+  uint32_t r;
+  if (ns == n) {
+    r = (uint32_t)K;
+  } else {
+    const float e = (float)K * (float)ns / (float)n;
+    r = (uint32_t)min((float)ns, ceilf(e + 3.f * sqrtf(e) + 2.f));
+  }
+  uint32_t T0 = smin;
+  if (smin != smax) {
+    const int hb = 31 - __clz(smin ^ smax);
+    const int wlo = hb >= kWin - 1 ? hb - (kWin - 1) : 0;
+    const int nbins = 1 << (hb - wlo + 1);
+    const uint32_t mhi = hb >= 31 ? 0u : ~((2u << hb) - 1u);
+    for (int i = tid; i < nbins; i += kThreads) S.hist[i] = 0;
+    __syncthreads();
+    hist_add(S.hist, (ks >> wlo) & (uint32_t)(nbins - 1), live_s);
+    __syncthreads();
+    uint32_t above;
+    const int b = top_bin(S.hist, nbins, r, S, &above);
+    T0 = (smin & mhi) | ((uint32_t)b << wlo);
+  }
+
+  // ---- 2. candidates: keys >= T0, per warp over its segment, in index order
+  uint32_t cnt = 0;
+  for (int c0 = w_lo; c0 < w_hi; c0 += kBatch * 128) {
+    if (c0 != w_lo) load_batch(s, c0, w_hi, vec, v);
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i0 = c0 + u * 128 + 4 * lane;
+      const uint32_t k[4] = {float_key(v[u].x), float_key(v[u].y), float_key(v[u].z), float_key(v[u].w)};
+      const bool f[4] = {i0 < w_hi && k[0] >= T0, i0 + 1 < w_hi && k[1] >= T0, i0 + 2 < w_hi && k[2] >= T0,
+                         i0 + 3 < w_hi && k[3] >= T0};
+      append4(S, warp, cnt, k, i0, f);
+    }
+  }
+  if (lane == 0) S.wcnt[warp] = cnt > kCap ? kCap + 1 : cnt;
+  __syncthreads();
+  uint32_t total = 0;
+  bool overflow = false;
+  for (int w = 0; w < kWarps; ++w) {
+    total += S.wcnt[w];
+    overflow |= S.wcnt[w] > kCap;
+  }
+  if (overflow || total < (uint32_t)K) {  // block-uniform
+    topk_general(s, n, K, out, S.hist, S.wsum, S.wgt, S.weq, &S.bin, &S.above);
     return;
   }
-  if (rank == 0 && tid == 0) a.count[q] = K;
-  // ---- slice of this CTA: [lo, hi)
-  const int per_cta = (n + kCluster - 1) / kCluster;
-  const int lo = min(n, rank * per_cta), hi = min(n, lo + per_cta);
-  const int m = hi - lo;
-  uint32_t kmin = 0xffffffffu, kmax = 0u;
-  for (int i0 = tid; i0 < m; i0 += kCThreads * kUnroll) {  // kUnroll independent loads in flight
-    uint32_t kv[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int i = i0 + u * kCThreads;
-      kv[u] = i < m ? float_key(__ldg(s + lo + i)) : 0u;
-    }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int i = i0 + u * kCThreads;
-      if (i < m) {
-        keys[i] = kv[u];
-        kmin = min(kmin, kv[u]);
-        kmax = max(kmax, kv[u]);
-      }
-    }
+  const uint32_t mycnt = S.wcnt[warp];
+  const uint32_t* ck = S.ckey[warp];
+  const uint32_t* ci = S.cidx[warp];
+  const uint32_t mr = (mycnt + 31) & ~31u;
+
+  // ---- 3. exact select among the candidates
+  uint32_t cmin = 0xffffffffu, cmax = 0u;
+  for (uint32_t j = lane; j < mycnt; j += 32) {
+    cmin = min(cmin, ck[j]);
+    cmax = max(cmax, ck[j]);
   }
-  kmin = __reduce_min_sync(0xffffffffu, kmin);
-  kmax = __reduce_max_sync(0xffffffffu, kmax);
-  if (lane == 0) {
-    wsum[warp] = kmin;
-    hist[warp] = kmax;
+  block_minmax(cmin, cmax, S.red);
+  uint32_t T = cmin, M = 0xffffffffu, remaining = (uint32_t)K;
+  int hb = cmin == cmax ? -1 : 31 - __clz(cmin ^ cmax);
+  if (hb >= 0) {
+    M = hb >= 31 ? 0u : ~((2u << hb) - 1u);
+    T = cmin & M;
   }
-  __syncthreads();
-  if (tid == 0) {
-    uint32_t mn = 0xffffffffu, mx = 0u;
-    for (int w = 0; w < kCWarps; ++w) {
-      mn = min(mn, wsum[w]);
-      mx = max(mx, hist[w]);
-    }
-    pub[0] = mn;
-    pub[1] = mx;
-  }
-  cluster.sync();
-  kmin = 0xffffffffu;
-  kmax = 0u;
-  for (int r = 0; r < kCluster; ++r) {
-    const uint32_t* rp = cluster.map_shared_rank(pub, r);
-    kmin = min(kmin, rp[0]);
-    kmax = max(kmax, rp[1]);
-  }
-  // ---- radix select over the bits where the keys differ
-  uint32_t prefix = kmin, remaining = (uint32_t)K;
-  int hb = kmin == kmax ? -1 : 31 - __clz(kmin ^ kmax);
-  if (hb >= 0) prefix &= (hb >= 31) ? 0u : ~((2u << hb) - 1u);
   while (hb >= 0) {
     const int wlo = hb >= kWin - 1 ? hb - (kWin - 1) : 0;
-    const uint32_t nbins = 1u << (hb - wlo + 1);
-    const uint32_t hmask = (hb >= 31) ? 0u : ~((2u << hb) - 1u);
-    for (int i = tid; i < (int)nbins; i += kCThreads) hist[i] = 0;
+    const int nbins = 1 << (hb - wlo + 1);
+    for (int i = tid; i < nbins; i += kThreads) S.hist[i] = 0;
     __syncthreads();
-    for (int i0 = tid; i0 < ((m + 31) & ~31); i0 += kCThreads) {
-      const bool live0 = i0 < m;
-      const uint32_t key = live0 ? keys[i0] : 0u;
-      hist_add(hist, (key >> wlo) & (nbins - 1), live0 && (key & hmask) == (prefix & hmask));
+    for (uint32_t j = lane; j < mr; j += 32) {
+      const uint32_t key = j < mycnt ? ck[j] : 0u;
+      hist_add(S.hist, (key >> wlo) & (uint32_t)(nbins - 1), j < mycnt && (key & M) == T);
     }
-    cluster.sync();  // every slice histogram complete
-    // reduce-scatter + all-gather: this CTA sums bins [rank * nbins / 8, ...) over
-    // the 8 slices and writes the sums into every CTA's merged histogram
-    {
-      const int span = (int)nbins / kCluster > 0 ? (int)nbins / kCluster : 1;
-      const int b0 = rank * span;
-      for (int bin = b0 + tid; bin < min((int)nbins, b0 + span); bin += kCThreads) {
-        uint32_t v[kCluster];
-#pragma unroll
-        for (int r = 0; r < kCluster; ++r) v[r] = cluster.map_shared_rank(hist, r)[bin];  // independent loads
-        uint32_t sum = 0;
-#pragma unroll
-        for (int r = 0; r < kCluster; ++r) sum += v[r];
-#pragma unroll
-        for (int r = 0; r < kCluster; ++r) cluster.map_shared_rank(merged, r)[bin] = sum;
-      }
-      if ((int)nbins < kCluster) {  // tiny windows: rank 0 alone
-        if (rank == 0)
-          for (int bin = tid; bin < (int)nbins; bin += kCThreads) {
-            uint32_t sum = 0;
-            for (int r = 0; r < kCluster; ++r) sum += cluster.map_shared_rank(hist, r)[bin];
-            for (int r = 0; r < kCluster; ++r) cluster.map_shared_rank(merged, r)[bin] = sum;
-          }
-      }
-    }
-    cluster.sync();  // merged histogram complete everywhere; slice histograms free
+    __syncthreads();
     uint32_t above;
-    const int b = cluster_find_bin(merged, (int)nbins, remaining, wsum, &s_bin, &s_above, &above);
-    prefix |= (uint32_t)b << wlo;
+    const int b = top_bin(S.hist, nbins, remaining, S, &above);
+    const uint32_t in_bin = S.hist[b];
     remaining -= above;
+    T |= (uint32_t)b << wlo;
+    M |= (uint32_t)(nbins - 1) << wlo;
+    __syncthreads();
+    if (remaining == in_bin) break;  // the whole bin is kept: its order does not matter
     hb = wlo - 1;
   }
-  const uint32_t T = prefix;          // the K-th largest key
-  const uint32_t need_eq = remaining;  // keys equal to T to keep, lowest index first
-  // ---- ordered output.  Per 32-key word: counts of keys > T and == T (ballots)
-  const int words = (m + 31) >> 5;
-  const uint32_t lt = (1u << lane) - 1u;
-  for (int w = warp; w < words; w += kCWarps) {
-    const int i = (w << 5) + lane;
-    const uint32_t k = i < m ? keys[i] : 0u;
-    const uint32_t gt = __ballot_sync(0xffffffffu, i < m && k > T);
-    const uint32_t eq = __ballot_sync(0xffffffffu, i < m && k == T);
-    if (lane == 0) {
-      wgt_cnt[w] = __popc(gt);
-      weq_cnt[w] = __popc(eq);
-    }
-  }
-  __syncthreads();
-  // slice totals, published for the higher-ranked CTAs
-  uint32_t g_loc = tid < words ? wgt_cnt[tid] : 0u, e_loc = tid < words ? weq_cnt[tid] : 0u;
-  uint32_t e_pre;
-  const uint32_t e_tot = block_exclusive(e_loc, wsum, &e_pre);
-  uint32_t g_pre;
-  const uint32_t g_tot = block_exclusive(g_loc, wsum, &g_pre);
-  if (tid == 0) {
-    pub[2] = g_tot;
-    pub[3] = e_tot;
-  }
-  cluster.sync();
-  uint32_t eq_before = 0, sel_before = 0;
-  for (int r = 0; r < rank; ++r) {
-    const uint32_t* rp = cluster.map_shared_rank(pub, r);
-    const uint32_t take_eq = need_eq > eq_before ? min(need_eq - eq_before, rp[3]) : 0u;
-    sel_before += rp[2] + take_eq;
-    eq_before += rp[3];
-  }
-  cluster.sync();  // remote reads of pub done before any CTA exits
-  // per word: ties before it (index order), keys it keeps, and its first output slot
-  uint32_t eqb = eq_before + e_pre;
-  const uint32_t take_w = tid < words ? (need_eq > eqb ? min(need_eq - eqb, e_loc) : 0u) + g_loc : 0u;
-  uint32_t sel_pre;
-  block_exclusive(take_w, wsum, &sel_pre);
-  if (tid < words) {
-    weq_cnt[tid] = eqb;                    // ties before this word
-    wgt_cnt[tid] = sel_before + sel_pre;   // first output slot of this word
-  }
-  __syncthreads();
-  for (int w = warp; w < words; w += kCWarps) {
-    const int i = (w << 5) + lane;
-    const uint32_t k = i < m ? keys[i] : 0u;
-    const bool is_gt = i < m && k > T;
-    const bool is_eq = i < m && k == T;
-    const uint32_t eq = __ballot_sync(0xffffffffu, is_eq);
-    const bool take = is_gt || (is_eq && weq_cnt[w] + __popc(eq & lt) < need_eq);
-    const uint32_t tk = __ballot_sync(0xffffffffu, take);
-    if (take) out[wgt_cnt[w] + __popc(tk & lt)] = lo + i;
-  }
-}
+  const uint32_t need = remaining;  // keys equal to T (under M) to keep, lowest index first
 
-// Rows longer than the cluster path holds: one CTA per such query.
-__global__ void __launch_bounds__(kThreads) topk_long_kernel(TopkArgs a) {
-  __shared__ uint32_t hist[4096];
-  __shared__ uint32_t wsum[kWarps];
-  __shared__ uint32_t wgt[kWarps], weq[kWarps];
-  __shared__ int s_bin;
-  __shared__ uint32_t s_above;
-  const int q = blockIdx.x;
-  const int p = a.q_pos[q];
-  int64_t nb = p >= 0 ? (int64_t)(p + 1) / kRatio : 0;
-  if (nb > a.ld) nb = a.ld;
-  if (a.K == 0 || nb <= kMaxFast) return;  // handled by the cluster kernel
-  topk_general(a.scores + (size_t)q * a.ld, (int)nb, a.K, a.sel + (size_t)q * a.K, hist, wsum, wgt, weq, &s_bin,
-               &s_above);
+  // ---- 4. ordered output
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t g = 0, e = 0;
+  for (uint32_t j = lane; j < mr; j += 32) {
+    const uint32_t k = j < mycnt ? ck[j] & M : 0u;
+    g += __popc(__ballot_sync(0xffffffffu, j < mycnt && k > T));
+    e += __popc(__ballot_sync(0xffffffffu, j < mycnt && k == T));
+  }
+  if (lane == 0) {
+    S.wgt[warp] = g;
+    S.weq[warp] = e;
+  }
+  __syncthreads();
+  if (warp == 0) {  // warp totals -> ties before each warp, first output slot of each warp
+    const uint32_t ew = S.weq[lane], gw = S.wgt[lane];
+    uint32_t einc = ew;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xffffffffu, einc, d);
+      if (lane >= d) einc += x;
+    }
+    const uint32_t eqb = einc - ew;
+    const uint32_t take = gw + (need > eqb ? min(need - eqb, ew) : 0u);
+    uint32_t tinc = take;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xffffffffu, tinc, d);
+      if (lane >= d) tinc += x;
+    }
+    S.weqb[lane] = eqb;
+    S.wslot[lane] = tinc - take;
+  }
+  __syncthreads();
+  uint32_t eqb = S.weqb[warp], slot = S.wslot[warp];
+  for (uint32_t j = lane; j < mr; j += 32) {
+    const uint32_t k = j < mycnt ? ck[j] & M : 0u;
+    const bool is_gt = j < mycnt && k > T;
+    const bool is_eq = j < mycnt && k == T;
+    const uint32_t eqm = __ballot_sync(0xffffffffu, is_eq);
+    const bool keep = is_gt || (is_eq && eqb + __popc(eqm & lt) < need);
+    const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+    if (keep) out[slot + __popc(kb & lt)] = (int32_t)ci[j];
+    slot += __popc(kb);
+    eqb += __popc(eqm);
+  }
 }
 
 }  // namespace
@@ -451,15 +468,12 @@ extern "C" int qsa_topk_blocks(const float* scores, int64_t scores_ld, const int
   if (nq < 0 || k < 0 || k > QSA_MAX_TOPK || scores_ld < 1) return QSA_ERR_INVALID_ARG;
   if (nq == 0) return QSA_OK;
   if (!scores || !q_pos || !count || (k > 0 && !sel)) return QSA_ERR_INVALID_ARG;
-  TopkArgs a{scores, scores_ld, q_pos, k, kMaxFast, sel, count, dev_status};
-  const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSliceCap * 4) != cudaSuccess) {
+  TopkArgs a{scores, scores_ld, q_pos, k, 0, sel, count, dev_status};
+  const int smem = (int)sizeof(TopkSmem);
+  if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
     (void)cudaGetLastError();
     return QSA_ERR_CUDA;
   }
-  topk_kernel<<<(unsigned)((int64_t)nq * kCluster), kCThreads, kSliceCap * 4, st>>>(a);
-  int rc = qsa_host::launch_status();
-  if (rc != QSA_OK) return rc;
-  if (scores_ld > kMaxFast) topk_long_kernel<<<(unsigned)nq, kThreads, 0, st>>>(a);
+  topk_kernel<<<(unsigned)nq, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(a);
   return qsa_host::launch_status();
 }

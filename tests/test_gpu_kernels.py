@@ -183,6 +183,52 @@ def test_topk_all_ties_take_lowest_indices():
     assert dec.sel[0].tolist() == list(range(100))
 
 
+def _topk_rows(kind, n, gen):
+    if kind == "random":
+        return torch.randn(n, generator=gen) * 100
+    if kind == "ascending":
+        return torch.arange(n, dtype=torch.float32) * 0.5
+    if kind == "descending":
+        return -torch.arange(n, dtype=torch.float32)
+    if kind == "ties":          # few distinct values: ties straddle the K-th key
+        return torch.randint(0, 7, (n,), generator=gen).float()
+    if kind == "neg_inf":       # blocks whose page was rejected score -inf
+        x = torch.randn(n, generator=gen)
+        x[torch.rand(n, generator=gen) < 0.5] = float("-inf")
+        return x
+    if kind == "hot_tail":      # the best blocks crowd into the last 5% of the row
+        x = torch.randn(n, generator=gen)
+        x[int(0.95 * n):] += 50
+        return x
+    raise ValueError(kind)
+
+
+@pytest.mark.parametrize("kind", ["random", "ascending", "descending", "ties", "neg_inf", "hot_tail"])
+@pytest.mark.parametrize("n,k,pad", [(513, 512, 0), (1024, 512, 3), (1025, 1, 0), (4095, 2048, 1),
+                                     (32768, 512, 0), (65536, 512, 5), (100000, 512, 0)])
+def test_topk_rows_match_oracle_on_every_path(kind, n, k, pad):
+    """Sampled-threshold path (random rows) and its fallback (sorted rows, heavy
+    ties, crowded tails overflow a warp's candidate list), aligned and
+    misaligned row strides, -inf scores, rows of 513 .. 100,000 blocks."""
+    gen = torch.Generator().manual_seed(n * 7 + k + pad)
+    rows = [_topk_rows(kind, n, gen), _topk_rows("random", n, gen)]
+    ld = n + pad
+    scores = torch.full((len(rows), ld), float("nan"), dtype=torch.float32)
+    for i, r in enumerate(rows):
+        scores[i, :n] = r
+    q_pos = torch.full((len(rows),), 4 * n - 1, dtype=torch.int32, device="cuda")
+    sel = torch.full((len(rows), k), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(len(rows), dtype=torch.int32, device="cuda")
+    st = _status()
+    qsa.qsa_topk_blocks(scores.cuda(), q_pos, k, sel, cnt, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for i, r in enumerate(rows):
+        ref = O.select_blocks(r.double().numpy(), k)
+        assert int(cnt[i]) == len(ref)
+        assert np.array_equal(sel[i].cpu().numpy()[:len(ref)], ref), f"{kind} row {i}"
+
+
 # ---------------------------------------------------------------- attention
 
 
