@@ -312,16 +312,38 @@ def run_native(args, rank, ws, local):
                                 stream=stream)]
     calls += dec.bind(inp["q"], inp["q_idx"], inp["w"], inp["q_seq"], inp["q_pos"], stream=stream)
 
+    def flush_l2():
+        # write 512 MiB, then read 256 MiB, so L2 is left holding clean lines
+        # (dirty flush lines would otherwise be written back inside the next
+        # timed step)
+        flush.zero_()
+        flush_sink.copy_(flush_read.sum())
+
     def between():
-        # L2 flush: write 512 MiB, then read 256 MiB so L2 is left holding clean
-        # lines (dirty flush lines would otherwise be written back inside the
-        # next timed step)
         with torch.cuda.stream(stream):
             cache.kc_partial.copy_(saved_partial)
-            flush.zero_()
-            flush_sink.copy_(flush_read.sum())
+            flush_l2()
+
+    def graph_of(fns, reps=1):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(reps):
+                for f in fns:
+                    f()
+        return g
+
+    def replay_ms(g):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1)
 
     # eager warm-up through the bound calls, then the step as one CUDA graph
+    # (no timing events inside it: an event between two kernels costs the GPU
+    # several microseconds)
     for _ in range(max(3, args.warmup)):
         for call in calls:
             call()
@@ -330,27 +352,23 @@ def run_native(args, rank, ws, local):
     status = int(st.item())
     if status:
         raise RuntimeError(f"device status {qsa.dev_status_names(status)}")
-    graph = qsa.StepGraph(calls, stream, timing=True)
+    graph = qsa.StepGraph(calls, stream)
     for _ in range(max(3, args.warmup)):
         graph.replay()
         between()
     torch.cuda.synchronize()
 
-    step_ms, kern = [], {n: [] for n in names}
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     barrier(ws)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         wall0 = time.perf_counter()
         for i in range(args.steps):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             torch.cuda.nvtx.range_push("qsa_step")   # lets a profiler select the timed launches
-            e0.record(stream)
+            evs[i][0].record(stream)
             graph.replay()
-            e1.record(stream)
+            evs[i][1].record(stream)
             torch.cuda.nvtx.range_pop()
-            for n, ms in zip(names, graph.kernel_ms()):   # waits for this step
-                kern[n].append(ms)
-            step_ms.append(e0.elapsed_time(e1))
             between()
         torch.cuda.synchronize()
         wall = time.perf_counter() - wall0
@@ -358,10 +376,29 @@ def run_native(args, rank, ws, local):
     status = int(st.item())
     if status:
         raise RuntimeError(f"device status after the timed steps: {qsa.dev_status_names(status)}")
-    kern_ms = {n: statistics.mean(v) for n, v in kern.items()}
+    step_ms = [a.elapsed_time(b) for a, b in evs]
     mean_ms = statistics.mean(step_ms)
     total_ms = max_over_ranks(sum(step_ms), ws)
     value = ws * wl.nq * args.steps / (total_ms / 1000.0)
+
+    # ---- per-kernel device time, cold L2: a graph of R x (flush, kernel) minus
+    # a graph of R x flush, divided by R
+    reps = 8
+    g_flush = graph_of([flush_l2], reps)
+    kern_ms = {}
+    for n, call in zip(names, calls):
+        g_k = graph_of([flush_l2, call], reps)
+        for _ in range(2):
+            replay_ms(g_k)
+            replay_ms(g_flush)
+        t_k = min(replay_ms(g_k) for _ in range(5))
+        t_f = min(replay_ms(g_flush) for _ in range(5))
+        kern_ms[n] = max(t_k - t_f, 1e-6) / reps
+        between()
+    torch.cuda.synchronize()
+    status = int(st.item())
+    if status:
+        raise RuntimeError(f"device status after the kernel timing: {qsa.dev_status_names(status)}")
 
     # ---- e2e: pinned host buffers, H2D of the step's inputs + the step (graph) + D2H of out/lse
     keys = ["k_new", "v_new", "kidx_new", "seq_id", "pos", "q", "q_idx", "w", "q_seq", "q_pos"]
@@ -415,6 +452,7 @@ def run_native(args, rank, ws, local):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {**wl.describe(), "l2": "flushed between timed steps (512 MiB write, then 256 MiB read); inputs also larger than L2",
                    "step": "append_kv + index_scores + topk_blocks + sparse_decode + combine, one CUDA graph",
+                   "kernel_timing": "per kernel: CUDA events around a graph of 8 x (L2 flush, kernel) minus one of 8 x (L2 flush), / 8",
                    "parallelism": f"dp{ws} (independent replicas)" if ws > 1 else "single GPU",
                    "chunk_units": dec.chunk_units, "max_splits": dec.max_splits},
         "hbm": {"pipeline_alg_bytes": ab["pipeline_spec"], "achieved_gbs": round(pipeline_gbs, 1), "peak_gbs": peak,
