@@ -208,8 +208,8 @@ def kernel_source_sha(kernel: str) -> str:
 
 
 def profiled_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current source of that kernel."""
+    """DRAM bytes per launch from the committed ncu summary of that kernel on
+    that workload, if it was taken on the kernel's current source."""
     p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(p):
         return None
@@ -441,7 +441,7 @@ def run_native(args, rank, ws, local):
     dom = max(names, key=lambda n: kern_ms[n])
     dom_key = {"topk": "topk"}.get(dom, dom)
     achieved = ab[dom_key] / (kern_ms[dom] / 1000.0) / 1e9
-    traffic = profiled_traffic(dom, args.workload)
+    traffic = profiled_traffic(dom, wl.name)
     kernels = {n: {"ms": round(kern_ms[n], 5), "alg_bytes": ab[n],
                    "gbs": round(ab[n] / (kern_ms[n] / 1000.0) / 1e9, 1)} for n in names}
     pipeline_gbs = ab["pipeline_spec"] / (mean_ms / 1000.0) / 1e9

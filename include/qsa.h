@@ -196,7 +196,7 @@ QSA_API int qsa_decode_plan(int32_t nq, int32_t hkv, int32_t k, int32_t target_c
  * chunk_units >= 1, max_splits >= the value qsa_decode_plan reports for
  * (k, chunk_units), scale > 0 (the pages keep the D256 scale 1/16).
  * The kernel gathers each selected micro-block (4 K rows + 4 V rows of one KV
- * head: one contiguous 4 KiB run) with one bulk async copy into shared memory
+ * head: one contiguous 4 KiB run) with 16-byte async copies into shared memory
  * and runs QK^T and PV on the tensor cores with fp32 accumulation; the
  * softmax weights P enter PV as a BF16 hi + lo pair (about 17 significant
  * bits), so short token sets keep full accuracy.
