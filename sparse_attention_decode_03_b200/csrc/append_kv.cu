@@ -66,6 +66,8 @@ __device__ __forceinline__ float4 block_sum(const AppendArgs& a, int64_t tok, in
 }
 
 __global__ void __launch_bounds__(kWarps * 32) append_scatter_kernel(AppendArgs a) {
+  pdl_launch_dependents();
+  pdl_wait_previous();
   const int lane = threadIdx.x & 31;
   const int64_t tok = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
   if (tok >= a.n) return;
@@ -110,6 +112,8 @@ __global__ void __launch_bounds__(kWarps * 32) append_scatter_kernel(AppendArgs 
 }
 
 __global__ void __launch_bounds__(kWarps * 32) append_partial_kernel(AppendArgs a) {
+  pdl_launch_dependents();
+  pdl_wait_previous();  // every read of the old open-block sums (scatter kernel) is done
   const int lane = threadIdx.x & 31;
   const int64_t tok = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
   if (tok >= a.n) return;
@@ -152,9 +156,7 @@ extern "C" int qsa_append_kv(const qsa_cache_t* cache, const void* k_new, const 
                dev_status};
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   const unsigned grid = (unsigned)((n + kWarps - 1) / kWarps);
-  append_scatter_kernel<<<grid, kWarps * 32, 0, s>>>(a);
-  int rc = qsa_host::launch_status();
+  int rc = qsa_host::launch(append_scatter_kernel, dim3(grid), dim3(kWarps * 32), 0, s, a);
   if (rc != QSA_OK) return rc;
-  append_partial_kernel<<<grid, kWarps * 32, 0, s>>>(a);
-  return qsa_host::launch_status();
+  return qsa_host::launch(append_partial_kernel, dim3(grid), dim3(kWarps * 32), 0, s, a);
 }

@@ -20,6 +20,8 @@ constexpr int kThreads = kHeadDim / 4;  // 64: four output dims per thread
 __global__ void __launch_bounds__(kThreads) combine_kernel(const float* __restrict__ part_o,
                                                            const float* __restrict__ part_lse, int S, int hq,
                                                            __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+  pdl_launch_dependents();
+  pdl_wait_previous();
   const int qh = blockIdx.x;
   const int q = qh / hq, h = qh % hq;
   const int tid = threadIdx.x;
@@ -66,7 +68,6 @@ extern "C" int qsa_combine(const float* part_o, const float* part_lse, int32_t n
   if ((reinterpret_cast<uintptr_t>(part_o) & 15u) || (reinterpret_cast<uintptr_t>(out) & 7u)) return QSA_ERR_INVALID_ARG;
   const int64_t grid = (int64_t)nq * hq;
   if (grid > 0x7fffffff) return QSA_ERR_UNSUPPORTED;
-  combine_kernel<<<(unsigned)grid, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      part_o, part_lse, max_splits, hq, static_cast<__nv_bfloat16*>(out), lse);
-  return qsa_host::launch_status();
+  return qsa_host::launch(combine_kernel, dim3((unsigned)grid), dim3(kThreads), 0, static_cast<cudaStream_t>(stream),
+                          part_o, part_lse, max_splits, hq, static_cast<__nv_bfloat16*>(out), lse);
 }

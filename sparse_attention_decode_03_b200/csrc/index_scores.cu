@@ -41,6 +41,8 @@ struct ScoreArgs {
 __device__ __forceinline__ float relu(float x) { return x > 0.f ? x : 0.f; }
 
 __global__ void __launch_bounds__(kWarps * 32) index_scores_kernel(ScoreArgs a) {
+  pdl_launch_dependents();
+  pdl_wait_previous();
   const int q = blockIdx.x / a.chunks_per_query;
   const int chunk = blockIdx.x % a.chunks_per_query;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -155,6 +157,6 @@ extern "C" int qsa_index_scores(const qsa_cache_t* cache, const void* q_idx, con
   a.st = dev_status;
   const int64_t grid = (int64_t)nq * a.chunks_per_query;
   if (grid > 0x7fffffff) return QSA_ERR_UNSUPPORTED;
-  index_scores_kernel<<<(unsigned)grid, kWarps * 32, 0, static_cast<cudaStream_t>(stream)>>>(a);
-  return qsa_host::launch_status();
+  return qsa_host::launch(index_scores_kernel, dim3((unsigned)grid), dim3(kWarps * 32), 0,
+                          static_cast<cudaStream_t>(stream), a);
 }

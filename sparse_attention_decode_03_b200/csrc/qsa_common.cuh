@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/qsa.h"
 
 #define QSA_DEVINL __device__ __forceinline__
@@ -160,6 +162,14 @@ QSA_DEVINL uint64_t l2_policy_evict_first() {
   return p;
 }
 
+// Programmatic dependent launch.  Every library kernel is launched so that the
+// next kernel on the stream may start while it runs: a kernel first lets its
+// dependents be scheduled, then waits until the previous kernel on the stream
+// has finished and its writes are visible, before it reads or writes any
+// buffer that kernel touches.  Outside such a launch both are no-ops.
+QSA_DEVINL void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+QSA_DEVINL void pdl_wait_previous() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 QSA_DEVINL void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -174,6 +184,27 @@ QSA_DEVINL uint32_t float_key(float f) {
 
 // host-side helpers
 namespace qsa_host {
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel on `stream` finishes (it waits for it on the device).
+template <typename... KArgs, typename... Args>
+inline int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QSA_ERR_CUDA;
+  }
+  return QSA_OK;
+}
+
 inline int launch_status() {
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;

@@ -663,6 +663,7 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
 
 __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
+  pdl_launch_dependents();
   const int64_t x0 = (int64_t)blockIdx.x * a.chunk;
   const int64_t x1 = min(x0 + a.chunk, a.total_slots);
   if (threadIdx.x == 0) {
@@ -678,6 +679,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(DecodeArgs a
     *reinterpret_cast<volatile int*>(smem + kOffAbort) = 0;
     fence_mbar_init();
   }
+  pdl_wait_previous();  // the selection and counts come from the previous kernel
   __syncthreads();
   if (x0 >= x1) return;
   const int warp = threadIdx.x >> 5;
@@ -742,6 +744,6 @@ extern "C" int qsa_sparse_decode(const qsa_cache_t* cache, const void* q, int32_
     (void)cudaGetLastError();
     return QSA_ERR_CUDA;
   }
-  sparse_decode_kernel<<<(unsigned)grid, kThreads, kSmemBytes, static_cast<cudaStream_t>(stream)>>>(a);
-  return qsa_host::launch_status();
+  return qsa_host::launch(sparse_decode_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes,
+                          static_cast<cudaStream_t>(stream), a);
 }

@@ -286,6 +286,8 @@ __device__ __forceinline__ void append4(TopkSmem& S, int warp, uint32_t& cnt, co
 }
 
 __global__ void __launch_bounds__(kThreads, 1) topk_kernel(TopkArgs a) {
+  pdl_launch_dependents();
+  pdl_wait_previous();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   TopkSmem& S = *reinterpret_cast<TopkSmem*>(smem_raw);
   const int q = blockIdx.x;
@@ -474,6 +476,6 @@ extern "C" int qsa_topk_blocks(const float* scores, int64_t scores_ld, const int
     (void)cudaGetLastError();
     return QSA_ERR_CUDA;
   }
-  topk_kernel<<<(unsigned)nq, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(a);
-  return qsa_host::launch_status();
+  return qsa_host::launch(topk_kernel, dim3((unsigned)nq), dim3(kThreads), (size_t)smem,
+                          static_cast<cudaStream_t>(stream), a);
 }
