@@ -167,6 +167,31 @@ def test_index_scores_and_topk_bit_exact(name, lengths, k):
         assert np.all(sel[row, cnt[row]:] == -1)
 
 
+@pytest.mark.parametrize("lengths,new,k", [
+    ([700, 2900, 33], 37, 64),     # 111 queries: ragged last tile, tiles spanning two sequences
+    ([9000], 20, 512),             # rows longer than one CTA's 2,048-block chunk
+])
+def test_query_tiled_index_scores_bit_exact(lengths, new, k):
+    """Chunked-prefill calls (many queries per sequence) take the query-tiled
+    indexer; its scores and the selections must match the oracle exactly."""
+    wl = C.shrink(C.get("prefill"), lengths, new_tokens=new, page_perm=True, k_top=k)
+    assert wl.nq >= 8 * wl.batch and wl.nq >= 16
+    cache, dec, st = run_step(wl, k=k)
+    assert st == 0
+    sc = dec.scores.cpu().numpy()
+    sel = dec.sel.cpu().numpy()
+    cnt = dec.count.cpu().numpy()
+    for row in range(wl.nq):
+        d = R.query_inputs(wl, row)
+        nb, _ = O.visible(d["p"])
+        kc = O.compress_keys(R.kidx_seq(wl, d["seq"], d["p"] + 1))
+        s_ref = O.block_scores(d["q_idx"], d["w"], kc)
+        assert np.array_equal(sc[row, :nb], s_ref.astype(np.float32)), f"scores row {row}"
+        sel_ref = O.select_blocks(s_ref, k)
+        assert cnt[row] == len(sel_ref)
+        assert np.array_equal(sel[row, :cnt[row]], sel_ref), f"selection row {row}"
+
+
 def test_topk_all_ties_take_lowest_indices():
     wl = C.shrink(C.get("quarter"), [2000], k_top=100)
     cache = H.new_cache(wl)
