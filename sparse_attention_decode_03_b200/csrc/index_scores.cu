@@ -128,22 +128,13 @@ __global__ void __launch_bounds__(kWarps * 32) index_scores_kernel(ScoreArgs a) 
 // Query-tiled variant for calls with many queries per sequence (chunked
 // prefill / extend): the queries of one sequence all read the same side cache,
 // so the work is a dense contraction [queries x 8 heads] x 128 x [blocks] and
-// a CTA of 16 consecutive queries reads each kc tile once for all of them.
-// Warp w holds, for the whole kernel, the A fragments of its 16 rows (queries
-// 2w and 2w+1, 8 heads each); 128-block kc tiles stream through a 3-stage
-// shared-memory ring (16-byte cp.async, rows padded to 272 B so the 16-byte
-// fragment reads are bank-conflict free); per 8-block n-tile: 8 mma.sync, then
-// w * ReLU and the sum over the 8 heads by a 3-step butterfly across the lanes.
-// Queries of the tile that belong to other sequences are handled by further
-// passes over their own pages (one pass per distinct sequence of the tile).
+// a CTA of 16 consecutive queries reads each 128-block kc tile once for all of
+// them.  Queries of a CTA that belong to different sequences are handled by
+// one pass per distinct sequence.
 
 constexpr int kTQ = 16;                   // queries per CTA
 constexpr int kTB = 128;                  // blocks per kc tile
-constexpr int kTStages = 3;
-constexpr int kTRow = kIdxDim * 2 + 16;   // 272 B: padded kc row in shared memory
-constexpr int kTTileBytes = kTB * kTRow;
-constexpr int kTChunkBlocks = 2048;       // blocks per CTA (gridDim.y splits longer rows)
-constexpr int kTSmem = kTStages * kTTileBytes + kTStages * kTB + 4 * kTQ * 4 + 64;
+constexpr int kTChunkBlocks = 8192;       // blocks per CTA (gridDim.y splits longer rows)
 
 struct TiledArgs {
   const __nv_bfloat16* kc;
@@ -159,7 +150,7 @@ struct TiledArgs {
   int32_t* st;
 };
 
-__device__ __forceinline__ void cp_async16_zfill_skip(uint32_t dst, const void* src) {
+__device__ __forceinline__ void cp_async16_cg(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
@@ -168,20 +159,140 @@ __device__ __forceinline__ void cp_async_wait_group() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-__global__ void __launch_bounds__(kWarps * 32, 2) index_scores_tiled_kernel(TiledArgs a) {
+// ---------------------------------------------------------------------------
+// The contraction runs on the 5th-generation tensor cores (tcgen05): per
+// 128-block kc tile, D[block][query*8 + head] = kc[block] .
+// q_idx[query][head] for the CTA's 16 queries, accumulated in tensor memory
+// (M = 128 blocks, N = 128, K = 128 dims in 8 steps of 16).  One TMEM lane per
+// block, so the w * ReLU head sum of a (query, block) score stays inside one
+// thread and the score stores are coalesced.
+//   warps 0-3  epilogue: tcgen05.ld of TMEM lanes 32w..32w+31, head sums, stores
+//   warp 4     TMEM allocation (512 columns: four accumulator buffers) and the
+//              MMA issue (one elected thread), tcgen05.commit to mbarriers
+//   warps 5-8  producers: 16-byte cp.async of q_idx (once) and of every kc
+//              tile into the canonical K-major, no-swizzle operand layout
+//              (8-row x 16-byte core matrices; the two 8-element halves of a
+//              16-element K step 128 B apart, 8-row groups 256 B apart), then
+//              a proxy fence and an mbarrier arrival per tile (a tile is
+//              published once the copies of the tile two later are issued,
+//              so three tiles are in flight per thread; 5-stage ring)
+// All waits are bounded; on expiry the CTA records QSA_DEV_TIMEOUT, stops
+// issuing work, drains what it issued and frees its tensor memory.
+
+constexpr int kUStages = 5;
+constexpr int kUTileBytes = kTB * kIdxDim * 2;                 // 32 KiB: one operand of 128 rows
+constexpr int kUEpiWarps = 4, kUMmaWarp = 4, kUProdWarp0 = 5, kUProdWarps = 4;
+constexpr int kUThreads = (kUProdWarp0 + kUProdWarps) * 32;    // 288
+constexpr int kUProdThreads = kUProdWarps * 32;
+constexpr int kUAcc = 4;                                       // accumulator buffers in tensor memory
+constexpr int kUTmemCols = kUAcc * 128;
+constexpr int kUOffB = 0;                                      // q_idx operand (128 rows)
+constexpr int kUOffA = kUOffB + kUTileBytes;                   // kc ring
+constexpr int kUOffW = kUOffA + kUStages * kUTileBytes;        // [16][8] weights
+constexpr int kUOffMeta = kUOffW + kTQ * kIdxHeads * 4;        // t_seq[16], t_nb[16], t_list[16], count, tmem, abort
+constexpr int kUOffBar = (kUOffMeta + (3 * kTQ + 4) * 4 + 7) & ~7;
+constexpr int kUNumBars = 2 * kUStages + 2 * kUAcc + 2;        // full/empty per stage, acc full/empty, b_full, done
+constexpr int kUSmem = kUOffBar + kUNumBars * 8;
+constexpr uint32_t kUIdesc = (1u << 4)                       // D: fp32
+                           | (1u << 7) | (1u << 10)          // A, B: bf16
+                           | ((uint32_t)(128 >> 3) << 17)    // N = 128
+                           | ((uint32_t)(128 >> 4) << 24);   // M = 128
+constexpr uint64_t kUWaitNs = 2000000000ull;
+
+// byte offset of 16-byte chunk c (dims 8c .. 8c+7) of operand row r
+__device__ __forceinline__ uint32_t umma_off(int r, int c) {
+  return (uint32_t)((c >> 1) * 4096 + (r >> 3) * 256 + (c & 1) * 128 + (r & 7) * 16);
+}
+
+// shared-memory matrix descriptor: K-major, no swizzle, LBO 128 B, SBO 256 B
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)(128u >> 4) << 16;
+  d |= (uint64_t)(256u >> 4) << 32;
+  d |= (uint64_t)1u << 46;  // descriptor version for sm_100
+  return d;
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+      ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0), "r"(0), "r"(0), "r"(0));
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// bounded mbarrier wait shared by all roles; false once the CTA aborted
+__device__ __forceinline__ bool uwait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* st) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 255u) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > kUWaitNs) {
+        flag(st, QSA_DEV_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kUThreads, 1) index_scores_umma_kernel(TiledArgs a) {
   pdl_launch_dependents();
-  pdl_wait_previous();
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint8_t* badrow = smem + kTStages * kTTileBytes;                           // [stage][128]
-  int32_t* t_seq = reinterpret_cast<int32_t*>(badrow + kTStages * kTB);      // [16] sequence of each query (-1: none)
-  int32_t* t_nb = t_seq + kTQ;                                               // [16] visible blocks
-  int32_t* t_list = t_nb + kTQ;                                              // [16] distinct sequences
-  int32_t* t_cnt = t_list + kTQ;                                             // [1]  how many
+  extern __shared__ __align__(128) uint8_t usmem[];
+  uint8_t* smem = usmem;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, t = lane & 3;
+  int32_t* t_seq = reinterpret_cast<int32_t*>(smem + kUOffMeta);
+  int32_t* t_nb = t_seq + kTQ;
+  int32_t* t_list = t_nb + kTQ;
+  int32_t* t_cnt = t_list + kTQ;
+  uint32_t* t_tmem = reinterpret_cast<uint32_t*>(t_cnt + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(t_cnt + 2);
+  float* t_w = reinterpret_cast<float*>(smem + kUOffW);
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t bar0 = sb + kUOffBar;
+  const uint32_t bar_full = bar0, bar_empty = bar0 + kUStages * 8;
+  const uint32_t bar_accf = bar0 + 2 * kUStages * 8, bar_acce = bar_accf + kUAcc * 8;
+  const uint32_t bar_bfull = bar_acce + kUAcc * 8, bar_done = bar_bfull + 8;
   const int q0 = blockIdx.x * kTQ;
   const int64_t blk_lo = (int64_t)blockIdx.y * kTChunkBlocks;
 
+  if (tid == 0) {
+    for (int i = 0; i < kUStages; ++i) {
+      mbar_init(bar_full + i * 8, kUProdThreads);
+      mbar_init(bar_empty + i * 8, 1);
+    }
+    for (int i = 0; i < kUAcc; ++i) {
+      mbar_init(bar_accf + i * 8, 1);
+      mbar_init(bar_acce + i * 8, kUEpiWarps * 32);
+    }
+    mbar_init(bar_bfull, kUProdThreads);
+    mbar_init(bar_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kUMmaWarp) {  // tensor memory for two 128 x 128 fp32 accumulators
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(t_tmem)),
+                 "r"(kUTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  pdl_wait_previous();
   if (tid < kTQ) {
     const int q = q0 + tid;
     int seq = -1, nb = 0;
@@ -203,6 +314,10 @@ __global__ void __launch_bounds__(kWarps * 32, 2) index_scores_tiled_kernel(Tile
     t_seq[tid] = seq;
     t_nb[tid] = nb;
   }
+  if (tid < kTQ * kIdxHeads) {
+    const int q = q0 + tid / kIdxHeads;
+    t_w[tid] = q < a.nq ? a.w[(size_t)q * kIdxHeads + tid % kIdxHeads] : 0.f;
+  }
   __syncthreads();
   if (tid == 0) {
     int n = 0;
@@ -215,111 +330,168 @@ __global__ void __launch_bounds__(kWarps * 32, 2) index_scores_tiled_kernel(Tile
     }
     *t_cnt = n;
   }
-
-  // A fragments: rows g -> (query 2w, head g), g + 8 -> (query 2w + 1, head g);
-  // chunk 4i + t of each 128-dim row (the contraction index permuted as in B)
-  const int qa = q0 + 2 * warp, qb = qa + 1;
-  uint4 fa[4], fb[4];
-  float wa = 0.f, wb = 0.f;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    fa[i] = qa < a.nq ? ldg_nc(a.q_idx + ((size_t)qa * kIdxHeads + g) * kIdxDim + (4 * i + t) * 8) : make_uint4(0, 0, 0, 0);
-    fb[i] = qb < a.nq ? ldg_nc(a.q_idx + ((size_t)qb * kIdxHeads + g) * kIdxDim + (4 * i + t) * 8) : make_uint4(0, 0, 0, 0);
-  }
-  if (qa < a.nq) wa = a.w[qa * kIdxHeads + g];
-  if (qb < a.nq) wb = a.w[qb * kIdxHeads + g];
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *t_tmem;
   const int nseq = *t_cnt;
-  const uint32_t ring = smem_u32(smem);
 
-  for (int si = 0; si < nseq; ++si) {
+  // the (sequence pass, tile) order every role walks
+  auto pass_range = [&](int si, int64_t& B0, int64_t& B1) {
     const int S = t_list[si];
     int nb_max = 0;
     for (int i = 0; i < kTQ; ++i)
       if (t_seq[i] == S) nb_max = max(nb_max, t_nb[i]);
-    const int64_t B0 = blk_lo, B1 = min((int64_t)nb_max, blk_lo + kTChunkBlocks);
-    if (B0 >= B1) continue;  // uniform
-    const int ntile = (int)((B1 - B0 + kTB - 1) / kTB);
-    const bool mine_a = qa < a.nq && t_seq[2 * warp] == S;
-    const bool mine_b = qb < a.nq && t_seq[2 * warp + 1] == S;
-    const int nb_a = t_nb[2 * warp], nb_b = t_nb[2 * warp + 1];
+    B0 = blk_lo;
+    B1 = min((int64_t)nb_max, blk_lo + kTChunkBlocks);
+  };
 
-    auto load_tile = [&](int j) {
-      const int stage = j % kTStages;
-      const int64_t b0 = B0 + (int64_t)j * kTB;
-#pragma unroll
-      for (int k = 0; k < (kTB * 16) / (kWarps * 32); ++k) {  // 8 x 16 B per thread
-        const int e = tid + k * kWarps * 32;
-        const int r = e >> 4, c = e & 15;
-        const int64_t b = b0 + r;
-        const uint32_t dst = ring + stage * kTTileBytes + r * kTRow + c * 16;
-        bool bad = false;
-        if (b < B1) {
-          const int phys = a.bt[(int64_t)S * a.mpps + b / kBlocksPerPage];
-          if (phys >= 0 && phys < a.num_pages) {
-            cp_async16_zfill_skip(dst, a.kc + ((size_t)phys * kBlocksPerPage + b % kBlocksPerPage) * kIdxDim + c * 8);
-          } else {
-            bad = true;
-            sts128(dst, make_uint4(0, 0, 0, 0));
-          }
-        } else {
-          sts128(dst, make_uint4(0, 0, 0, 0));
-        }
-        if (c == 0) {
-          badrow[stage * kTB + r] = bad ? 1 : 0;
-          if (bad) flag(a.st, QSA_DEV_BAD_PAGE);
-        }
-      }
-    };
-
-#pragma unroll
-    for (int j = 0; j < kTStages - 1; ++j) {
-      if (j < ntile) load_tile(j);
-      cp_async_commit();
+  if (warp >= kUProdWarp0) {
+    // ---------------- producers
+    const int pt = tid - kUProdWarp0 * 32;  // 0..127
+    // q_idx operand: row = query * 8 + head, 16 chunks of 16 B
+    for (int e = pt; e < kTQ * kIdxHeads * 16; e += kUProdThreads) {
+      const int r = e >> 4, c = e & 15;
+      const int q = q0 + (r >> 3);
+      const uint32_t dst = sb + kUOffB + umma_off(r, c);
+      if (q < a.nq)
+        cp_async16_cg(dst, a.q_idx + ((size_t)q * kIdxHeads + (r & 7)) * kIdxDim + c * 8);
+      else
+        sts128(dst, make_uint4(0, 0, 0, 0));
     }
-    for (int j = 0; j < ntile; ++j) {
-      cp_async_wait_group<kTStages - 2>();
-      __syncthreads();  // tile j visible to all; every warp is done with tile j - 1
-      if (j + kTStages - 1 < ntile) load_tile(j + kTStages - 1);
-      cp_async_commit();
-      const int stage = j % kTStages;
-      const uint32_t tile = ring + stage * kTTileBytes;
-      const int64_t b0 = B0 + (int64_t)j * kTB;
-      if (!mine_a && !mine_b) continue;
-#pragma unroll 2
-      for (int nt = 0; nt < kTB / 8; ++nt) {
-        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+    cp_async_commit();
+    cp_async_wait_group<0>();
+    fence_async_smem();
+    mbar_arrive(bar_bfull);
+    int j = 0;  // global tile counter
+    int pend0 = -1, pend1 = -1;  // tiles whose copies are in flight and not yet signalled (older first)
+    for (int si = 0; si < nseq && !*abort_flag; ++si) {
+      int64_t B0, B1;
+      pass_range(si, B0, B1);
+      const int S = t_list[si];
+      for (int64_t b0 = B0; b0 < B1; b0 += kTB, ++j) {
+        const int stage = j % kUStages;
+        if (j >= kUStages && !uwait(bar_empty + stage * 8, (uint32_t)((j / kUStages - 1) & 1), abort_flag, a.st))
+          break;
+        const uint32_t tile = sb + kUOffA + stage * kUTileBytes;
+        // this thread's 16 chunks: chunk c = pt % 16 of rows pt / 16 + 8k; their page ids are
+        // loaded first, all together (the copies below are compiler barriers)
+        constexpr int kPer = kTB * 16 / kUProdThreads;  // 16
+        const int c = pt & 15;
+        int phys[kPer];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint4 kb = lds128(tile + (nt * 8 + g) * kTRow + (4 * i + t) * 16);
-          float(&acc)[4] = (i & 1) ? s1 : s0;
-          mma_bf16_16816(acc, fa[i].x, fb[i].x, fa[i].y, fb[i].y, kb.x, kb.y);
-          mma_bf16_16816(acc, fa[i].z, fb[i].z, fa[i].w, fb[i].w, kb.z, kb.w);
+        for (int k = 0; k < kPer; ++k) {
+          const int64_t b = b0 + (pt >> 4) + 8 * k;
+          phys[k] = b < B1 ? __ldg(a.bt + (int64_t)S * a.mpps + b / kBlocksPerPage) : -1;
         }
-        // (row g | g + 8, block 2t | 2t + 1) -> w * ReLU, then the sum over the 8 heads
-        const float v0 = wa * relu(s0[0] + s1[0]), v1 = wa * relu(s0[1] + s1[1]);
-        const float v2 = wb * relu(s0[2] + s1[2]), v3 = wb * relu(s0[3] + s1[3]);
-        const bool up4 = (g & 4) != 0, up2 = (g & 2) != 0;
-        float x0 = up4 ? v2 : v0, x1 = up4 ? v3 : v1;
-        x0 += __shfl_xor_sync(0xffffffffu, up4 ? v0 : v2, 16);
-        x1 += __shfl_xor_sync(0xffffffffu, up4 ? v1 : v3, 16);
-        float z = up2 ? x1 : x0;
-        z += __shfl_xor_sync(0xffffffffu, up2 ? x0 : x1, 8);
-        z += __shfl_xor_sync(0xffffffffu, z, 4);
-        // lanes with g even hold query (g & 4 ? qb : qa), block nt * 8 + 2t + (g >> 1 & 1)
-        if ((g & 1) == 0) {
-          const int r = nt * 8 + 2 * t + ((g >> 1) & 1);
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+          const int r = (pt >> 4) + 8 * k;
           const int64_t b = b0 + r;
-          const bool for_b = up4;
-          const int q = for_b ? qb : qa;
-          const int nbq = for_b ? nb_b : nb_a;
-          if ((for_b ? mine_b : mine_a) && b < nbq)
-            a.scores[(size_t)q * a.ld + b] = badrow[stage * kTB + r] ? -INFINITY : z;
+          const uint32_t dst = tile + umma_off(r, c);
+          if (b < B1 && phys[k] >= 0 && phys[k] < a.num_pages) {
+            cp_async16_cg(dst, a.kc + ((size_t)phys[k] * kBlocksPerPage + b % kBlocksPerPage) * kIdxDim + c * 8);
+          } else {
+            sts128(dst, make_uint4(0, 0, 0, 0));
+            if (b < B1 && c == 0) flag(a.st, QSA_DEV_BAD_PAGE);
+          }
         }
+        cp_async_commit();
+        if (pend0 >= 0) {  // the copies of the tile issued two tiles ago have landed: publish it
+          cp_async_wait_group<2>();
+          fence_async_smem();
+          mbar_arrive(bar_full + (pend0 % kUStages) * 8);
+        }
+        pend0 = pend1;
+        pend1 = j;
       }
     }
     cp_async_wait_group<0>();
-    __syncthreads();  // the ring is free before the next sequence's pass
+    fence_async_smem();
+    if (pend0 >= 0) mbar_arrive(bar_full + (pend0 % kUStages) * 8);
+    if (pend1 >= 0) mbar_arrive(bar_full + (pend1 % kUStages) * 8);
+  } else if (warp == kUMmaWarp) {
+    // ---------------- MMA issue (one thread)
+    if (lane == 0) {
+      bool ok = uwait(bar_bfull, 0, abort_flag, a.st);
+      const uint64_t bdesc0 = umma_desc(sb + kUOffB);
+      int j = 0;
+      for (int si = 0; si < nseq && ok; ++si) {
+        int64_t B0, B1;
+        pass_range(si, B0, B1);
+        for (int64_t b0 = B0; b0 < B1 && ok; b0 += kTB, ++j) {
+          const int stage = j % kUStages, acc = j % kUAcc;
+          if (!uwait(bar_full + stage * 8, (uint32_t)((j / kUStages) & 1), abort_flag, a.st)) { ok = false; break; }
+          if (j >= kUAcc && !uwait(bar_acce + acc * 8, (uint32_t)((j / kUAcc - 1) & 1), abort_flag, a.st)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc0 = umma_desc(sb + kUOffA + stage * kUTileBytes);
+#pragma unroll
+          for (int ks = 0; ks < kIdxDim / 16; ++ks)  // 4096 B per 16-element K step, in 16-B units
+            umma_f16(tmem + acc * 128, adesc0 + (uint64_t)(ks * 256), bdesc0 + (uint64_t)(ks * 256), kUIdesc,
+                     ks > 0 ? 1u : 0u);
+          umma_commit(bar_empty + stage * 8);  // the kc stage is free once these MMAs finish
+          umma_commit(bar_accf + acc * 8);     // the accumulator is ready
+        }
+      }
+      umma_commit(bar_done);  // every MMA issued above has completed when this fires
+      mbar_wait_bounded(bar_done, 0, kUWaitNs);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue: row = block b0 + 32 * warp + lane
+    const int row = 32 * warp + lane;
+    int j = 0;
+    for (int si = 0; si < nseq; ++si) {
+      int64_t B0, B1;
+      pass_range(si, B0, B1);
+      const int S = t_list[si];
+      for (int64_t b0 = B0; b0 < B1; b0 += kTB, ++j) {
+        const int acc = j % kUAcc;
+        const int64_t b = b0 + row;
+        // a block on a rejected page scores -inf (its kc rows were zero-filled)
+        const int phys = b < B1 ? a.bt[(int64_t)S * a.mpps + b / kBlocksPerPage] : 0;
+        if (!uwait(bar_accf + acc * 8, (uint32_t)((j / kUAcc) & 1), abort_flag, a.st)) goto epi_done;
+        tc_fence_after();
+        float sc[kTQ];
+        const uint32_t taddr = tmem + acc * 128 + ((uint32_t)(32 * warp) << 16);
+#pragma unroll
+        for (int h8 = 0; h8 < kTQ / 8; ++h8) {  // 4 loads of two queries (16 columns) each, then one wait
+          uint32_t r[4][16];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) tmem_ld16(taddr + (h8 * 4 + u) * 16, r[u]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              const int ql = 2 * (h8 * 4 + u) + k;
+              float s = 0.f;
+#pragma unroll
+              for (int hd = 0; hd < kIdxHeads; ++hd)
+                s += t_w[ql * kIdxHeads + hd] * relu(__uint_as_float(r[u][8 * k + hd]));
+              sc[ql] = s;
+            }
+        }
+        tc_fence_before();
+        mbar_arrive(bar_acce + acc * 8);  // this thread is done reading the accumulator
+        const bool bad = b < B1 && (phys < 0 || phys >= a.num_pages);
+#pragma unroll
+        for (int ql = 0; ql < kTQ; ++ql) {
+          if (t_seq[ql] == S && b < t_nb[ql])
+            a.scores[(size_t)(q0 + ql) * a.ld + b] = bad ? -INFINITY : sc[ql];
+        }
+      }
+    }
+  epi_done:;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kUMmaWarp) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kUTmemCols) : "memory");
   }
 }
 
@@ -369,13 +541,13 @@ extern "C" int qsa_index_scores(const qsa_cache_t* cache, const void* q_idx, con
     const int64_t gy = (max_blocks + kTChunkBlocks - 1) / kTChunkBlocks;
     const int64_t gx = ((int64_t)nq + kTQ - 1) / kTQ;
     if (gy > 65535 || gx > 0x7fffffff) return QSA_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(index_scores_tiled_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTSmem) !=
+    if (cudaFuncSetAttribute(index_scores_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kUSmem) !=
         cudaSuccess) {
       (void)cudaGetLastError();
       return QSA_ERR_CUDA;
     }
-    return qsa_host::launch(index_scores_tiled_kernel, dim3((unsigned)gx, (unsigned)gy), dim3(kWarps * 32),
-                            (size_t)kTSmem, static_cast<cudaStream_t>(stream), t);
+    return qsa_host::launch(index_scores_umma_kernel, dim3((unsigned)gx, (unsigned)gy), dim3(kUThreads),
+                            (size_t)kUSmem, static_cast<cudaStream_t>(stream), t);
   }
   // the most kc pages any query can see is the block-table width
   int64_t max_pages = cache->max_pages_per_seq;

@@ -169,7 +169,7 @@ def test_index_scores_and_topk_bit_exact(name, lengths, k):
 
 @pytest.mark.parametrize("lengths,new,k", [
     ([700, 2900, 33], 37, 64),     # 111 queries: ragged last tile, tiles spanning two sequences
-    ([9000], 20, 512),             # rows longer than one CTA's 2,048-block chunk
+    ([36000], 20, 512),            # rows longer than one CTA's 8,192-block chunk
 ])
 def test_query_tiled_index_scores_bit_exact(lengths, new, k):
     """Chunked-prefill calls (many queries per sequence) take the query-tiled
