@@ -44,7 +44,10 @@ Readings where the pages are silent (each is listed in the design notes):
     one pair's slots that falls in one chunk; an empty split has o = 0 and
     lse = -inf;
   * combine: lse = log sum_s exp(lse_s), o = sum_s exp(lse_s - lse) o_s; every
-    lse_s = -inf gives o = 0 exactly and lse = -inf.
+    lse_s = -inf gives o = 0 exactly and lse = -inf;
+  * the FP8 main K/V cache stores e4m3(K) and e4m3(V) of the BF16 rows (round
+    to nearest even, saturated, no scale); attention runs on those values and
+    the indexer side cache stays BF16.
 
 Every function below is pinned by tests in ``tests/test_oracle_pins.py``
 against closed forms, library routines or brute force; no function is
@@ -73,6 +76,35 @@ def bf16_round(x) -> np.ndarray:
     out = r.view(np.float32).copy()
     nan = np.isnan(a)
     out[nan] = np.nan
+    return out
+
+
+# ----------------------------------------------------------------------------
+# FP8 e4m3 (the optional FP8 main K/V cache)
+
+
+E4M3_MAX = 448.0   # largest finite e4m3 value: 1.75 * 2^8
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Round values to the nearest FP8 e4m3 value (ties to even), saturating
+    finite values beyond +-448 to +-448; returns fp64.
+
+    e4m3 ([BSS], section "Apa yang dikatakan oleh klaster patch di sekitarnya
+    tentang Qwen4Exp": the FP8 e4m3 main KV cache) has a sign, 4 exponent bits
+    with bias 7 and 3 mantissa bits: normal values (1 + m/8) * 2^(e-7) for
+    e in 1..15 (the all-ones code is NaN, no infinities), subnormal values
+    m * 2^-9.  Between 2^E and 2^(E+1) the grid step is 2^(E-3); below 2^-6 it
+    is 2^-9.  The quantisation carries no scale factor (scale 1)."""
+    a = np.asarray(x, dtype=np.float64)
+    mag = np.abs(a)
+    _, ex = np.frexp(mag)                     # mag = f * 2^ex, f in [0.5, 1)
+    E = np.maximum(ex - 1, -6)                # floor(log2 mag), subnormal range below 2^-6
+    step = np.ldexp(1.0, E - 3)
+    q = np.rint(mag / step) * step            # np.rint: round half to even
+    q = np.minimum(q, E4M3_MAX)
+    out = np.copysign(q, a)
+    out[np.isnan(a)] = np.nan
     return out
 
 

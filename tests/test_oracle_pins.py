@@ -34,6 +34,52 @@ def test_bf16_round_matches_torch_conversion():
     assert np.array_equal(np.isinf(got), np.isinf(ref))
 
 
+# ---------------------------------------------------------------- FP8 e4m3 rounding
+
+def _e4m3_code_values():
+    """The value of every non-NaN e4m3 code, decoded from its bit fields."""
+    vals = []
+    for code in range(256):
+        s, e, m = code >> 7, (code >> 3) & 15, code & 7
+        if e == 15 and m == 7:
+            continue  # NaN
+        v = (m / 8.0) * 2.0 ** -6 if e == 0 else (1 + m / 8.0) * 2.0 ** (e - 7)
+        vals.append(-v if s else v)
+    return np.array(vals)
+
+
+def test_e4m3_round_matches_torch_float8_conversion():
+    x = np.concatenate([
+        RNG.standard_normal(30000) * np.exp(RNG.uniform(-16, 7, 30000)),
+        RNG.uniform(-448, 448, 5000), [0.0, -0.0, 448.0, -448.0, 2.0 ** -9, 2.0 ** -10, 3 * 2.0 ** -10]])
+    x = x[np.abs(x) <= 448].astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(O.e4m3_round(x), ref)
+
+
+def test_e4m3_every_code_is_a_fixed_point():
+    v = _e4m3_code_values()
+    assert np.array_equal(O.e4m3_round(v), v)
+    u = np.unique(v)
+    assert u.size == 253 and u.max() == 448.0 and np.min(u[u > 0]) == 2.0 ** -9
+
+
+def test_e4m3_ties_to_even_and_saturation():
+    u = np.unique(_e4m3_code_values())
+    pos = u[u >= 0]
+    mid = (pos[:-1] + pos[1:]) / 2          # exact midpoints of neighbouring codes
+    got = O.e4m3_round(mid)
+    # the code with an even mantissa wins: its value / (grid step) is even
+    lo, hi = pos[:-1], pos[1:]
+    step = hi - lo
+    want = np.where(np.rint(lo / step) % 2 == 0, lo, hi)
+    assert np.array_equal(got, want)
+    assert np.array_equal(O.e4m3_round(-mid), -want)
+    sat = O.e4m3_round(np.array([448.5, 464.0, 479.0, 1e6, -1e30]))
+    assert np.array_equal(sat, [448.0, 448.0, 448.0, 448.0, -448.0])
+    assert np.isnan(O.e4m3_round(np.array([np.nan])))[0]
+
+
 # ---------------------------------------------------------------- compression
 
 def test_compress_keys_integer_sum_is_exact():
