@@ -46,7 +46,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", default="long", choices=list(C.ALL))
+    ap.add_argument("--workload", default="long", choices=list(C.ALL) + list(C.FP8))
     ap.add_argument("--batch", type=int, default=0, help="use only the first N sequences (profiling a small case)")
     ap.add_argument("--context", type=int, default=0, help="override every context length (profiling a small case)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -172,8 +172,9 @@ def algorithmic_bytes(wl: C.Workload, count: np.ndarray, q_pos: np.ndarray, spli
     nb = (q_pos.astype(np.int64) + 1) // 4
     t = (q_pos.astype(np.int64) + 1) % 4
     n_new = wl.batch * wl.new_tokens
-    tok_kv = wl.hkv * 256 * 2 * 2                       # K + V bytes of one token
-    append = n_new * (2 * tok_kv + 128 * 2)            # read new K/V/kidx, write K/V (+kc, small)
+    tok_in = wl.hkv * 256 * 2 * 2                       # K + V bytes of one new token (BF16 inputs)
+    tok_kv = wl.hkv * 256 * 2 * (1 if wl.kv_fp8 else 2)  # K + V bytes of one cached token
+    append = n_new * (tok_in + tok_kv + 128 * 2)       # read new K/V/kidx, write K/V (+kc, small)
     side = int(nb.sum()) * 128 * 2                      # kc rows read
     scores_w = int(nb.sum()) * 4
     index = side + scores_w
@@ -449,7 +450,7 @@ def run_native(args, rank, ws, local):
     line = {
         "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": mean_ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": "e4m3 kv + bf16" if wl.kv_fp8 else "bf16", "data": "synthetic",
         "config": {**wl.describe(), "l2": "flushed between timed steps (512 MiB write, then 256 MiB read); inputs also larger than L2",
                    "step": "append_kv + index_scores + topk_blocks + sparse_decode + combine, one CUDA graph",
                    "kernel_timing": "per kernel: CUDA events around a graph of 8 x (L2 flush, kernel) minus one of 8 x (L2 flush), / 8",

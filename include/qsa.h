@@ -86,18 +86,27 @@ typedef enum {
  * One cache group ([DCP]: the selector and the main KV cache are kept in one
  * cache group so they cannot drift apart).  The main K/V and the compressed
  * indexer side cache are paged by the SAME physical page ids.
- *   kv_pages    bf16 [num_pages][num_kv_heads][16][2][4][256]  post-RoPE K and V:
- *               per page and KV head, its 16 micro-blocks of 4 tokens, each
- *               holding the 4 K rows then the 4 V rows, so one selected
- *               micro-block of one KV head is a single contiguous 4 KiB run
+ *   kv_pages    [num_pages][num_kv_heads][16][2][4][256] elements of type
+ *               kv_dtype, post-RoPE K and V: per page and KV head, its 16
+ *               micro-blocks of 4 tokens, each holding the 4 K rows then the 4
+ *               V rows, so one selected micro-block of one KV head is a single
+ *               contiguous run (4 KiB in BF16, 2 KiB in FP8)
  *               (token t of a page: micro-block t / 4, row t % 4)
  *   kc_pages    bf16 [num_pages][16][128]  kc of the 16 micro-blocks of a page
  *   kc_partial  fp32 [max_seqs][128]       running fp32 sum of each sequence's
  *                                           open (incomplete) micro-block
  *   block_table int32 [max_seqs][max_pages_per_seq]  logical page -> physical page
+ *   kv_dtype    QSA_KV_BF16, or QSA_KV_FP8_E4M3: the main K/V stored as FP8
+ *               e4m3 (1 byte per element, the BF16 value rounded to nearest
+ *               even and saturated to +-448, no scale; the FP8 e4m3 main KV
+ *               cache of [BSS], section "Apa yang dikatakan oleh klaster patch
+ *               di sekitarnya tentang Qwen4Exp"), which halves the bytes the
+ *               sparse attention gathers.  The side cache stays BF16.
  * All buffers are caller-owned device memory; the library writes kv/kc pages
  * and kc_partial only in qsa_append_kv.
  */
+#define QSA_KV_BF16 0
+#define QSA_KV_FP8_E4M3 1
 typedef struct {
   void* kv_pages;
   void* kc_pages;
@@ -107,6 +116,7 @@ typedef struct {
   int32_t max_seqs;
   int32_t max_pages_per_seq;
   int32_t num_kv_heads;
+  int32_t kv_dtype;
 } qsa_cache_t;
 
 /* Human-readable name of a qsa_status value (static string). */
@@ -114,7 +124,7 @@ QSA_API const char* qsa_status_string(int status);
 
 /* ABI version of this header (bumped on any signature change). */
 QSA_API int qsa_abi_version(void);
-#define QSA_ABI_VERSION 2
+#define QSA_ABI_VERSION 3
 
 /*
  * qsa_append_kv -- write n new tokens into the cache group.
@@ -123,7 +133,8 @@ QSA_API int qsa_abi_version(void);
  * the QSA side caches: a token with seq_id < 0 is skipped entirely.
  *   k_new, v_new  bf16 [n][Hkv][256];  kidx_new  bf16 [n][128] (indexer keys)
  *   seq_id, pos   int32 [n]  sequence and absolute position of each token
- * Effect: K/V rows written at page block_table[seq][pos/64], token pos%64.  The
+ * Effect: K/V rows written at page block_table[seq][pos/64], token pos%64 (as
+ * e4m3, round to nearest even, saturated to +-448, when kv_dtype is FP8).  The
  * indexer keys of a micro-block are summed in fp32 in token order (continuing
  * kc_partial when the block began in an earlier call); when the token at
  * position 4j+3 arrives, kc_pages row j = BF16(sum) (round to nearest even).

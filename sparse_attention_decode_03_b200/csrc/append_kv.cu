@@ -35,6 +35,24 @@ struct AppendArgs {
   int32_t* st;
 };
 
+// 8 BF16 values -> 8 FP8 e4m3 (round to nearest even, saturated to +-448), as 8 bytes
+__device__ __forceinline__ uint2 bf16x8_to_e4m3x8(uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t out[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint16_t pr[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const uint32_t x = w[2 * h + k];  // two BF16: low half = first element
+      const float lo = __uint_as_float(x << 16), hi = __uint_as_float(x & 0xffff0000u);
+      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pr[k]) : "f"(hi), "f"(lo));  // first element -> low byte
+    }
+    out[h] = (uint32_t)pr[0] | ((uint32_t)pr[1] << 16);
+  }
+  return make_uint2(out[0], out[1]);
+}
+
 // Number of this call's tokens directly before `tok` that belong to the same
 // sequence at consecutive positions (at most `limit`).
 __device__ __forceinline__ int run_before(const AppendArgs& a, int64_t tok, int seq, int p, int limit) {
@@ -90,14 +108,22 @@ __global__ void __launch_bounds__(kWarps * 32) append_scatter_kernel(AppendArgs 
   }
   const int slot = p % kPage;
   const int hkv = a.c.num_kv_heads;
-  __nv_bfloat16* kv = static_cast<__nv_bfloat16*>(a.c.kv_pages);
   for (int h = 0; h < hkv; ++h) {
-    // [page][h][micro-block][K rows | V rows][256]
+    // [page][h][micro-block][K rows | V rows][256] elements
     const size_t blk = (((size_t)page * hkv + h) * kBlocksPerPage + slot / kRatio) * (2 * kRatio * kHeadDim);
     const size_t dst = blk + (size_t)(slot % kRatio) * kHeadDim + lane * 8;
     const size_t src = ((size_t)tok * hkv + h) * kHeadDim + lane * 8;
-    *reinterpret_cast<uint4*>(kv + dst) = *reinterpret_cast<const uint4*>(a.k_new + src);
-    *reinterpret_cast<uint4*>(kv + dst + kRatio * kHeadDim) = *reinterpret_cast<const uint4*>(a.v_new + src);
+    const uint4 kv8 = *reinterpret_cast<const uint4*>(a.k_new + src);
+    const uint4 vv8 = *reinterpret_cast<const uint4*>(a.v_new + src);
+    if (a.c.kv_dtype == QSA_KV_FP8_E4M3) {
+      uint8_t* kv = static_cast<uint8_t*>(a.c.kv_pages);
+      *reinterpret_cast<uint2*>(kv + dst) = bf16x8_to_e4m3x8(kv8);
+      *reinterpret_cast<uint2*>(kv + dst + kRatio * kHeadDim) = bf16x8_to_e4m3x8(vv8);
+    } else {
+      __nv_bfloat16* kv = static_cast<__nv_bfloat16*>(a.c.kv_pages);
+      *reinterpret_cast<uint4*>(kv + dst) = kv8;
+      *reinterpret_cast<uint4*>(kv + dst + kRatio * kHeadDim) = vv8;
+    }
   }
   if ((p & 3) == 3) {  // this token closes micro-block p / 4
     const int m = run_before(a, tok, seq, p, 3);
@@ -143,6 +169,7 @@ extern "C" int qsa_append_kv(const qsa_cache_t* cache, const void* k_new, const 
   if (!c.kv_pages || !c.kc_pages || !c.kc_partial || !c.block_table) return QSA_ERR_INVALID_ARG;
   if (!k_new || !v_new || !kidx_new || !seq_id || !pos) return QSA_ERR_INVALID_ARG;
   if (c.num_pages < 1 || c.max_seqs < 1 || c.max_pages_per_seq < 1 || c.num_kv_heads < 1) return QSA_ERR_INVALID_ARG;
+  if (c.kv_dtype != QSA_KV_BF16 && c.kv_dtype != QSA_KV_FP8_E4M3) return QSA_ERR_UNSUPPORTED;
   if (!aligned16(c.kv_pages) || !aligned16(c.kc_partial) || !aligned16(k_new) ||
       !aligned16(v_new) || (reinterpret_cast<uintptr_t>(c.kc_pages) & 7u) || (reinterpret_cast<uintptr_t>(kidx_new) & 7u))
     return QSA_ERR_INVALID_ARG;

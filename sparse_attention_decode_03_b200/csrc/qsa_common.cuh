@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -49,6 +50,12 @@ QSA_DEVINL uint4 lds128(uint32_t saddr) {
   return r;
 }
 
+QSA_DEVINL uint2 lds64(uint32_t saddr) {
+  uint2 r;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(saddr));
+  return r;
+}
+
 QSA_DEVINL void sts128(uint32_t saddr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(saddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
 }
@@ -65,6 +72,42 @@ QSA_DEVINL void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D(16x8 fp32) += A(16x16 fp16, row) * B(16x8 fp16, col)
+QSA_DEVINL void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                              uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Four FP8 e4m3 bytes (first element in the low byte) -> four FP16, exact
+// (every e4m3 value is an FP16 value): .x = elements 0, 1 and .y = 2, 3, each
+// with the lower-indexed element in the low half.
+QSA_DEVINL uint2 e4m3x4_to_f16x4(uint32_t b) {
+  uint2 r;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(r.x), "=r"(r.y)
+      : "r"(b));
+  return r;
+}
+
+// Eight e4m3 bytes -> eight FP16 laid out like eight BF16 loaded as a uint4.
+QSA_DEVINL uint4 e4m3x8_to_f16x8(uint2 v) {
+  const uint2 a = e4m3x4_to_f16x4(v.x), b = e4m3x4_to_f16x4(v.y);
+  return make_uint4(a.x, a.y, b.x, b.y);
+}
+
+// FP16x2 of (lo, hi), rounded to nearest even, finite values clamped to +-65504.
+QSA_DEVINL uint32_t pack_f16_sat(float lo, float hi) {
+  lo = fminf(fmaxf(lo, -65504.f), 65504.f);
+  hi = fminf(fmaxf(hi, -65504.f), 65504.f);
+  __half2 v = __floats2half2_rn(lo, hi);  // .x = lo (low half), .y = hi
+  return *reinterpret_cast<uint32_t*>(&v);
 }
 
 QSA_DEVINL uint32_t pack_bf16(float lo, float hi) {

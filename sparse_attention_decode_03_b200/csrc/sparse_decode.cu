@@ -53,32 +53,59 @@ constexpr int kConsumerThreads = kConsumerWarps * 32;
 // pair count and tile T owned by pair T % 4, that tile's owner is the pair that
 // consumed tile T, so no mbarrier wait can ever skip a phase (a parity wait can
 // only name the current phase or the one before it).
-constexpr int kStages = 8;
 constexpr int kUnitsPerTile = 4;
 constexpr int kBatch = 32;                                             // units per lookup batch
 constexpr int kRound = 4;                                              // lookup batches resolved together
 constexpr int kDescSlots = 2 * kRound;                                 // lookup batches in flight
-constexpr int kHalfBytes = kRatio * kHeadDim * 2;                      // 2048: 4 K (or V) rows
-constexpr int kUnitBytes = 2 * kHalfBytes;                             // 4096: K rows then V rows
-constexpr int kSlotStride = kUnitBytes + 32;                           // 4128: 16-B bank-group skew of 2
-constexpr int kStageBytes = kUnitsPerTile * kSlotStride;
 constexpr int kQRowStride = kHeadDim * 2 + 64;                         // 576
 constexpr int kQBufBytes = 16 * kQRowStride;
 constexpr int kCombRow = kHeadDim + 4;                                 // floats
 constexpr int kCombBytes = 2 * 16 * kCombRow * 4;                      // two warps' O
-constexpr int kOffRing = 0;
-constexpr int kOffQ = kOffRing + kStages * kStageBytes;
-constexpr int kOffComb = kOffQ + kQBufBytes;
-constexpr int kOffML = kOffComb + kCombBytes;
-constexpr int kOffDescOff = kOffML + kPairs * 16 * 2 * 4;
-constexpr int kOffDescRows = kOffDescOff + kDescSlots * kBatch * 8;
-constexpr int kOffMeta = kOffDescRows + kDescSlots * kBatch * 4;
-constexpr int kOffBar = (kOffMeta + kStages * 4 + 7) & ~7;
-constexpr int kNumBars = 2 * kStages + 2 * kDescSlots;
-constexpr int kOffAbort = kOffBar + kNumBars * 8;
-constexpr int kSmemBytes = kOffAbort + 16;
-static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kStages % kPairs == 0 && kStages % kCopyWarps == 0, "tile ownership must repeat with the stage ring");
+
+// Shared-memory layout for BF16 (F8 = false) or FP8 e4m3 (F8 = true) K/V.
+// A unit (one micro-block of one KV head) is 4 K rows then 4 V rows: 4 KiB in
+// BF16, 2 KiB in FP8; the FP8 ring has twice the stages for the same bytes.
+template <bool F8>
+struct Lay {
+  static constexpr int kStages = F8 ? 16 : 8;
+  static constexpr int kHalfBytes = kRatio * kHeadDim * (F8 ? 1 : 2);  // 4 K (or V) rows
+  static constexpr int kUnitBytes = 2 * kHalfBytes;
+  static constexpr int kSlotStride = kUnitBytes + 32;                  // 16-B bank-group skew of 2
+  static constexpr int kStageBytes = kUnitsPerTile * kSlotStride;
+  static constexpr int kOffRing = 0;
+  static constexpr int kOffQ = kOffRing + kStages * kStageBytes;
+  static constexpr int kOffComb = kOffQ + kQBufBytes;
+  static constexpr int kOffML = kOffComb + kCombBytes;
+  static constexpr int kOffDescOff = kOffML + kPairs * 16 * 2 * 4;
+  static constexpr int kOffDescRows = kOffDescOff + kDescSlots * kBatch * 8;
+  static constexpr int kOffMeta = kOffDescRows + kDescSlots * kBatch * 4;
+  static constexpr int kOffBar = (kOffMeta + kStages * 4 + 7) & ~7;
+  static constexpr int kNumBars = 2 * kStages + 2 * kDescSlots;
+  static constexpr int kOffAbort = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffAbort + 16;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kStages % kPairs == 0 && kStages % kCopyWarps == 0, "tile ownership must repeat with the stage ring");
+};
+
+#define QSA_DECODE_LAYOUT                                   \
+  using LY = Lay<F8>;                                       \
+  constexpr int kStages = LY::kStages;                      \
+  constexpr int kHalfBytes = LY::kHalfBytes;                \
+  constexpr int kUnitBytes = LY::kUnitBytes;                \
+  constexpr int kSlotStride = LY::kSlotStride;              \
+  constexpr int kStageBytes = LY::kStageBytes;              \
+  constexpr int kOffRing = LY::kOffRing;                    \
+  constexpr int kOffQ = LY::kOffQ;                          \
+  constexpr int kOffComb = LY::kOffComb;                    \
+  constexpr int kOffML = LY::kOffML;                        \
+  constexpr int kOffDescOff = LY::kOffDescOff;              \
+  constexpr int kOffDescRows = LY::kOffDescRows;            \
+  constexpr int kOffMeta = LY::kOffMeta;                    \
+  constexpr int kOffBar = LY::kOffBar;                      \
+  constexpr int kOffAbort = LY::kOffAbort;                  \
+  (void)kStages; (void)kHalfBytes; (void)kUnitBytes; (void)kSlotStride; (void)kStageBytes; (void)kOffRing; \
+  (void)kOffQ; (void)kOffComb; (void)kOffML; (void)kOffDescOff; (void)kOffDescRows; (void)kOffMeta;      \
+  (void)kOffBar; (void)kOffAbort
 // full barrier: the 32 lanes' copy-completion arrivals + the owning copy warp's
 // lane 0, whose plain (release) arrival publishes the stage's row mask
 constexpr int kFullArrivals = 33;
@@ -87,7 +114,7 @@ constexpr int kBarConsumers = 1;                  // named barrier id
 constexpr uint64_t kNoCopy = ~0ull;
 
 struct DecodeArgs {
-  const __nv_bfloat16* kv_pages;
+  const uint8_t* kv_bytes;
   const int32_t* bt;
   int32_t num_pages, max_seqs, mpps, hkv;
   const __nv_bfloat16* q;
@@ -225,7 +252,9 @@ __device__ __forceinline__ bool warp_aborted(volatile int* abort_flag) {
 // Resolves kRound batches per round: the selection loads of all of them are
 // issued together, then the page-table loads, so a round costs two dependent
 // global-load latencies for 4 x 32 units.
+template <bool F8>
 __device__ void lookup_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_t x1) {
+  QSA_DECODE_LAYOUT;
   const int lane = threadIdx.x & 31;
   uint64_t* d_off = reinterpret_cast<uint64_t*>(smem + kOffDescOff);
   uint32_t* d_rows = reinterpret_cast<uint32_t*>(smem + kOffDescRows);
@@ -298,7 +327,7 @@ __device__ void lookup_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int6
           flag(a.st, QSA_DEV_BAD_PAGE);
         } else {
           off = (((uint64_t)phys[r] * a.hkv + g[r]) * kBlocksPerPage + (uint64_t)(j[r] % kBlocksPerPage)) *
-                (2 * kRatio * kHeadDim);
+                kUnitBytes;  // bytes
           rows = lane < i_main[r] ? 0xFu : (1u << t[r]) - 1u;
         }
       }
@@ -311,7 +340,9 @@ __device__ void lookup_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int6
   }
 }
 
+template <bool F8>
 __device__ void copy_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_t x1, int cw) {
+  QSA_DECODE_LAYOUT;
   const int lane = threadIdx.x & 31;
   const uint32_t ring = smem_u32(smem + kOffRing);
   const uint32_t bar_full = smem_u32(smem + kOffBar);
@@ -323,7 +354,7 @@ __device__ void copy_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
   uint32_t* meta = reinterpret_cast<uint32_t*>(smem + kOffMeta);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
   const uint64_t policy = l2_policy_evict_first();
-  const char* kv = reinterpret_cast<const char*>(a.kv_pages);
+  const char* kv = reinterpret_cast<const char*>(a.kv_bytes);
   int64_t T = 0;
   BatchIter it;
   bool have = iter_begin(a, it, x0, x1);
@@ -355,7 +386,7 @@ __device__ void copy_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
       for (int u = 0; u < kUnitsPerTile; ++u) {
         const uint64_t uoff = __shfl_sync(0xffffffffu, off, (tb * kUnitsPerTile + u) & 31);
         if (tb * kUnitsPerTile + u < n_units && uoff != kNoCopy) {
-          const char* src = kv + uoff * sizeof(__nv_bfloat16) + lane * 16;
+          const char* src = kv + uoff + lane * 16;
 #pragma unroll
           for (int c = 0; c < kUnitBytes / 512; ++c) cp_async16(dst + u * kSlotStride + c * 512, src + c * 512, policy);
         }
@@ -392,7 +423,9 @@ __device__ __forceinline__ bool consumer_wait(const DecodeArgs& a, uint32_t bar,
   }
 }
 
+template <bool F8>
 __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_t x1) {
+  QSA_DECODE_LAYOUT;
   const int tid = threadIdx.x;  // 0..255
   const int warp = tid >> 5, lane = tid & 31;
   const int cp = warp >> 1;     // consumer pair: owns tiles T with T % 4 == cp
@@ -408,31 +441,41 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
   const int64_t n_slots = (int64_t)a.K + 1;
   const int G = a.G;
 
-  // K tile: S column n = gq of n-tile j is token (slot ks, row 2j + ke)
+  // K tile: S column n = gq of n-tile j is token (slot ks, row 2j + ke); the
+  // lane holds dims 32i + 8tq .. + 7 of it for k-step pair i (Q likewise)
+  constexpr int kRowBytes = kHalfBytes / kRatio;  // one K or V row: 512 B BF16, 256 B FP8
+  constexpr int kElt = kRowBytes / kHeadDim;
   const int ke = gq & 1;
   const int ks = ((gq >> 1) + 2 * ke) & 3;
-  const uint32_t k_off = ks * kSlotStride + ke * 512 + tq * 16;
+  const uint32_t k_off = ks * kSlotStride + ke * kRowBytes + tq * 8 * kElt;
   // S/P columns held by this lane: n = 2tq + e -> (slot (tq + 2e) & 3, row 2j + e)
   const int ps0 = tq, ps1 = (tq + 2) & 3;
   // V tokens of the PV B fragment: (ps0,row0) (ps1,row1) (ps0,row2) (ps1,row3); this
   // warp reads V chunks 8qq + gq for qq in {2 half, 2 half + 1}
-  const uint32_t vh = kHalfBytes + half * 256;
-  const uint32_t v_off0 = ps0 * kSlotStride + vh + 0 * 512 + gq * 16;
-  const uint32_t v_off1 = ps1 * kSlotStride + vh + 1 * 512 + gq * 16;
-  const uint32_t v_off2 = ps0 * kSlotStride + vh + 2 * 512 + gq * 16;
-  const uint32_t v_off3 = ps1 * kSlotStride + vh + 3 * 512 + gq * 16;
+  const uint32_t vh = kHalfBytes + half * 128 * kElt;
+  const uint32_t v_off0 = ps0 * kSlotStride + vh + 0 * kRowBytes + gq * 8 * kElt;
+  const uint32_t v_off1 = ps1 * kSlotStride + vh + 1 * kRowBytes + gq * 8 * kElt;
+  const uint32_t v_off2 = ps0 * kSlotStride + vh + 2 * kRowBytes + gq * 8 * kElt;
+  const uint32_t v_off3 = ps1 * kSlotStride + vh + 3 * kRowBytes + gq * 8 * kElt;
   const int vb0 = ps0 * 4 + 0, vb1 = ps1 * 4 + 1, vb2 = ps0 * 4 + 2, vb3 = ps1 * 4 + 3;
 
   int64_t T_base = 0;
   for (int64_t pair = x0 / n_slots; pair <= (x1 - 1) / n_slots; ++pair) {
     const Seg s = make_seg(a, pair, x0, x1, tid == 0);
     const uint32_t qb = smem_u32(smem + kOffQ);  // the merge barriers of the last segment order reuse
-    // ---- stage Q rows of this KV group (rows >= G are zero)
+    // ---- stage Q rows of this KV group (rows >= G are zero); FP8 K/V takes
+    // FP16 operands, so Q is converted (exact for normal BF16 values within +-65504)
     for (int idx = tid; idx < 16 * 32; idx += kConsumerThreads) {
       const int row = idx >> 5, c = idx & 31;
       uint4 v = make_uint4(0, 0, 0, 0);
       if (row < G && s.query_ok)
         v = ldg_nc(a.q + ((size_t)s.q * a.hq + (size_t)s.g * G + row) * kHeadDim + c * 8);
+      if constexpr (F8) {
+        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) w[e] = pack_f16_sat(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u));
+        v = make_uint4(w[0], w[1], w[2], w[3]);
+      }
       sts128(qb + row * kQRowStride + c * 16, v);
     }
     named_bar_sync(kBarConsumers, kConsumerThreads);
@@ -464,10 +507,16 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
         const uint4 qc = lds128(qb + (gq + 8) * kQRowStride + (4 * i + tq) * 16);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          const uint4 kk = lds128(kb + k_off + j * 1024 + i * 64);
           float(&acc)[4] = (i & 1) ? sb[j] : sa[j];
-          mma_bf16_16816(acc, qa.x, qc.x, qa.y, qc.y, kk.x, kk.y);
-          mma_bf16_16816(acc, qa.z, qc.z, qa.w, qc.w, kk.z, kk.w);
+          if constexpr (F8) {
+            const uint4 kk = e4m3x8_to_f16x8(lds64(kb + k_off + j * 2 * kRowBytes + i * 32));
+            mma_f16_16816(acc, qa.x, qc.x, qa.y, qc.y, kk.x, kk.y);
+            mma_f16_16816(acc, qa.z, qc.z, qa.w, qc.w, kk.z, kk.w);
+          } else {
+            const uint4 kk = lds128(kb + k_off + j * 2 * kRowBytes + i * 64);
+            mma_bf16_16816(acc, qa.x, qc.x, qa.y, qc.y, kk.x, kk.y);
+            mma_bf16_16816(acc, qa.z, qc.z, qa.w, qc.w, kk.z, kk.w);
+          }
         }
       }
       // ---- mask, online softmax (base-2 logits)
@@ -513,13 +562,22 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
           o[nt][3] *= al1;
         }
       }
-      // P = hi + lo, both BF16: the PV product keeps ~17 significant bits of
-      // every weight (BF16 alone, 8 bits, is too coarse for short token sets)
+      // BF16 K/V: P = hi + lo, both BF16, so the PV product keeps ~17
+      // significant bits of every weight (BF16 alone, 8 bits, is too coarse for
+      // short token sets).  FP8 K/V: P in FP16 (11 bits) against e4m3 V (4 bits).
       uint32_t pa[4], pl[4];
-      split_bf16(pr[0][0], pr[0][1], pa[0], pl[0]);
-      split_bf16(pr[0][2], pr[0][3], pa[1], pl[1]);
-      split_bf16(pr[1][0], pr[1][1], pa[2], pl[2]);
-      split_bf16(pr[1][2], pr[1][3], pa[3], pl[3]);
+      if constexpr (F8) {
+        pa[0] = pack_f16_sat(pr[0][0], pr[0][1]);
+        pa[1] = pack_f16_sat(pr[0][2], pr[0][3]);
+        pa[2] = pack_f16_sat(pr[1][0], pr[1][1]);
+        pa[3] = pack_f16_sat(pr[1][2], pr[1][3]);
+        pl[0] = pl[1] = pl[2] = pl[3] = 0u;
+      } else {
+        split_bf16(pr[0][0], pr[0][1], pa[0], pl[0]);
+        split_bf16(pr[0][2], pr[0][3], pa[1], pl[1]);
+        split_bf16(pr[1][0], pr[1][1], pa[2], pl[2]);
+        split_bf16(pr[1][2], pr[1][3], pa[3], pl[3]);
+      }
 
       // ---- O += P V for this warp's 128 dims: 16 n-tiles, k = the tile's 16 tokens
       const bool full = mask == 0xffffu;
@@ -527,10 +585,18 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
       const bool ok2 = (mask >> vb2) & 1u, ok3 = (mask >> vb3) & 1u;
 #pragma unroll
       for (int qh = 0; qh < 2; ++qh) {
-        uint4 x0v = lds128(kb + v_off0 + qh * 128);
-        uint4 x1v = lds128(kb + v_off1 + qh * 128);
-        uint4 x2v = lds128(kb + v_off2 + qh * 128);
-        uint4 x3v = lds128(kb + v_off3 + qh * 128);
+        uint4 x0v, x1v, x2v, x3v;
+        if constexpr (F8) {
+          x0v = e4m3x8_to_f16x8(lds64(kb + v_off0 + qh * 64));
+          x1v = e4m3x8_to_f16x8(lds64(kb + v_off1 + qh * 64));
+          x2v = e4m3x8_to_f16x8(lds64(kb + v_off2 + qh * 64));
+          x3v = e4m3x8_to_f16x8(lds64(kb + v_off3 + qh * 64));
+        } else {
+          x0v = lds128(kb + v_off0 + qh * 128);
+          x1v = lds128(kb + v_off1 + qh * 128);
+          x2v = lds128(kb + v_off2 + qh * 128);
+          x3v = lds128(kb + v_off3 + qh * 128);
+        }
         if (!full) {  // masked rows may hold stale or never-written data
           if (!ok0) x0v = make_uint4(0, 0, 0, 0);
           if (!ok1) x1v = make_uint4(0, 0, 0, 0);
@@ -547,10 +613,15 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
           const uint32_t hi01 = __byte_perm(a0[r], a1[r], 0x7632);
           const uint32_t lo23 = __byte_perm(a2[r], a3[r], 0x5410);
           const uint32_t hi23 = __byte_perm(a2[r], a3[r], 0x7632);
-          mma_bf16_16816(o[qh * 8 + 2 * r], pa[0], pa[1], pa[2], pa[3], lo01, lo23);
-          mma_bf16_16816(o[qh * 8 + 2 * r + 1], pa[0], pa[1], pa[2], pa[3], hi01, hi23);
-          mma_bf16_16816(o[qh * 8 + 2 * r], pl[0], pl[1], pl[2], pl[3], lo01, lo23);
-          mma_bf16_16816(o[qh * 8 + 2 * r + 1], pl[0], pl[1], pl[2], pl[3], hi01, hi23);
+          if constexpr (F8) {
+            mma_f16_16816(o[qh * 8 + 2 * r], pa[0], pa[1], pa[2], pa[3], lo01, lo23);
+            mma_f16_16816(o[qh * 8 + 2 * r + 1], pa[0], pa[1], pa[2], pa[3], hi01, hi23);
+          } else {
+            mma_bf16_16816(o[qh * 8 + 2 * r], pa[0], pa[1], pa[2], pa[3], lo01, lo23);
+            mma_bf16_16816(o[qh * 8 + 2 * r + 1], pa[0], pa[1], pa[2], pa[3], hi01, hi23);
+            mma_bf16_16816(o[qh * 8 + 2 * r], pl[0], pl[1], pl[2], pl[3], lo01, lo23);
+            mma_bf16_16816(o[qh * 8 + 2 * r + 1], pl[0], pl[1], pl[2], pl[3], hi01, hi23);
+          }
         }
       }
       __syncwarp();
@@ -661,7 +732,9 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
   }
 }
 
+template <bool F8>
 __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(DecodeArgs a) {
+  QSA_DECODE_LAYOUT;
   extern __shared__ __align__(128) uint8_t smem[];
   pdl_launch_dependents();
   const int64_t x0 = (int64_t)blockIdx.x * a.chunk;
@@ -684,11 +757,23 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(DecodeArgs a
   if (x0 >= x1) return;
   const int warp = threadIdx.x >> 5;
   if (warp >= kCopyWarp0 && warp < kCopyWarp0 + kCopyWarps)
-    copy_warp(a, smem, x0, x1, warp - kCopyWarp0);
+    copy_warp<F8>(a, smem, x0, x1, warp - kCopyWarp0);
   else if (warp == kLookupWarp)
-    lookup_warp(a, smem, x0, x1);
+    lookup_warp<F8>(a, smem, x0, x1);
   else
-    consumers(a, smem, x0, x1);
+    consumers<F8>(a, smem, x0, x1);
+}
+
+template <bool F8>
+int launch_decode(const DecodeArgs& a, int64_t grid, void* stream) {
+  constexpr int kSmem = Lay<F8>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(sparse_decode_kernel<F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QSA_ERR_CUDA;
+  }
+  return qsa_host::launch(sparse_decode_kernel<F8>, dim3((unsigned)grid), dim3(kThreads), kSmem,
+                          static_cast<cudaStream_t>(stream), a);
 }
 
 }  // namespace
@@ -707,6 +792,7 @@ extern "C" int qsa_sparse_decode(const qsa_cache_t* cache, const void* q, int32_
   if (c.num_kv_heads < 1 || hq % c.num_kv_heads != 0) return QSA_ERR_INVALID_ARG;
   if (hq / c.num_kv_heads > QSA_MAX_GROUP) return QSA_ERR_UNSUPPORTED;
   if (max_splits < qsa_splits_bound(k, chunk_units)) return QSA_ERR_INVALID_ARG;
+  if (c.kv_dtype != QSA_KV_BF16 && c.kv_dtype != QSA_KV_FP8_E4M3) return QSA_ERR_UNSUPPORTED;
   if (nq == 0) return QSA_OK;
   if (!c.kv_pages || !c.block_table || !q || !q_seq || !q_pos || !count || !part_o || !part_lse ||
       (k > 0 && !sel))
@@ -716,7 +802,7 @@ extern "C" int qsa_sparse_decode(const qsa_cache_t* cache, const void* q, int32_
        reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(part_o)) & 15u)
     return QSA_ERR_INVALID_ARG;
   DecodeArgs a;
-  a.kv_pages = static_cast<const __nv_bfloat16*>(c.kv_pages);
+  a.kv_bytes = static_cast<const uint8_t*>(c.kv_pages);
   a.bt = c.block_table;
   a.num_pages = c.num_pages;
   a.max_seqs = c.max_seqs;
@@ -739,11 +825,5 @@ extern "C" int qsa_sparse_decode(const qsa_cache_t* cache, const void* q, int32_
   a.st = dev_status;
   const int64_t grid = (a.total_slots + a.chunk - 1) / a.chunk;
   if (grid > 0x7fffffff) return QSA_ERR_UNSUPPORTED;
-  cudaError_t e = cudaFuncSetAttribute(sparse_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e != cudaSuccess) {
-    (void)cudaGetLastError();
-    return QSA_ERR_CUDA;
-  }
-  return qsa_host::launch(sparse_decode_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes,
-                          static_cast<cudaStream_t>(stream), a);
+  return c.kv_dtype == QSA_KV_FP8_E4M3 ? launch_decode<true>(a, grid, stream) : launch_decode<false>(a, grid, stream);
 }

@@ -42,7 +42,12 @@ class qsa_cache_t(ctypes.Structure):
     _fields_ = [("kv_pages", ctypes.c_void_p), ("kc_pages", ctypes.c_void_p),
                 ("kc_partial", ctypes.c_void_p), ("block_table", ctypes.c_void_p), ("num_pages", ctypes.c_int32),
                 ("max_seqs", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32),
-                ("num_kv_heads", ctypes.c_int32)]
+                ("num_kv_heads", ctypes.c_int32), ("kv_dtype", ctypes.c_int32)]
+
+
+KV_BF16 = 0
+KV_FP8_E4M3 = 1
+_KV_TORCH = {KV_BF16: torch.bfloat16, KV_FP8_E4M3: torch.float8_e4m3fn}
 
 
 def _load() -> ctypes.CDLL:
@@ -116,15 +121,19 @@ class PagedCache:
     side cache, paged by the same page ids, plus the per-sequence open-block sum.
 
     kv_pages is [page][Hkv][16 micro-blocks][2 (K, V)][4 rows][256]: one selected
-    micro-block of one KV head is a contiguous 4 KiB run."""
+    micro-block of one KV head is a contiguous run, 4 KiB in BF16 (kv_dtype
+    KV_BF16) or 2 KiB in FP8 e4m3 (KV_FP8_E4M3)."""
 
     def __init__(self, num_pages: int, max_seqs: int, max_pages_per_seq: int, num_kv_heads: int,
-                 block_table: torch.Tensor | None = None, device="cuda"):
+                 block_table: torch.Tensor | None = None, device="cuda", kv_dtype: int = KV_BF16):
         dev = torch.device(device)
+        if kv_dtype not in _KV_TORCH:
+            raise ValueError(f"kv_dtype must be KV_BF16 or KV_FP8_E4M3, got {kv_dtype}")
         self.num_pages, self.max_seqs, self.max_pages_per_seq, self.num_kv_heads = (
             int(num_pages), int(max_seqs), int(max_pages_per_seq), int(num_kv_heads))
+        self.kv_dtype = int(kv_dtype)
         self.kv_pages = torch.empty((num_pages, num_kv_heads, BLOCKS_PER_PAGE, 2, RATIO, HEAD_DIM),
-                                    dtype=torch.bfloat16, device=dev)
+                                    dtype=_KV_TORCH[self.kv_dtype], device=dev)
         self.kc_pages = torch.empty((num_pages, BLOCKS_PER_PAGE, IDX_DIM), dtype=torch.bfloat16, device=dev)
         self.kc_partial = torch.zeros((max_seqs, IDX_DIM), dtype=torch.float32, device=dev)
         if block_table is None:
@@ -137,7 +146,7 @@ class PagedCache:
         if self._struct is None:
             self._struct = qsa_cache_t(self.kv_pages.data_ptr(), self.kc_pages.data_ptr(),
                                        self.kc_partial.data_ptr(), self.block_table.data_ptr(), self.num_pages,
-                                       self.max_seqs, self.max_pages_per_seq, self.num_kv_heads)
+                                       self.max_seqs, self.max_pages_per_seq, self.num_kv_heads, self.kv_dtype)
         return self._struct
 
     def k_view(self) -> torch.Tensor:

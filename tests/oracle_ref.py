@@ -38,6 +38,8 @@ def kv_reader(wl: C.Workload, seq: int, prefix_from=None):
             t = torch.from_numpy(pos[m])
             K[m] = C.k_rows(wl, int(s), t).float().numpy()
             V[m] = C.v_rows(wl, int(s), t).float().numpy()
+        if wl.kv_fp8:  # the cache holds e4m3 of the BF16 rows
+            K, V = O.e4m3_round(K), O.e4m3_round(V)
         return K, V
     return rows
 

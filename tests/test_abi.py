@@ -25,7 +25,7 @@ def test_library_exports_every_declared_symbol():
     lib = ctypes.CDLL(qsa.LIB_PATH)
     for n in header_functions():
         assert hasattr(lib, n), n
-    assert qsa.ABI_VERSION == 2
+    assert qsa.ABI_VERSION == 3
     assert qsa.status_string(0) == "QSA_OK" and qsa.status_string(-3) == "QSA_ERR_CUDA"
 
 
@@ -65,6 +65,11 @@ def test_host_validation_returns_before_any_cuda_call():
     assert L.qsa_index_scores(cp, None, fake, fake, fake, 1, fake, 16, None, None) == -1
     assert L.qsa_combine(ctypes.c_void_p(0x1004), fake, 1, 4, 16, fake, fake, None) == -1  # misaligned
     assert L.qsa_combine(fake, fake, 1, 0, 16, fake, fake, None) == -1
+    # K/V storage types: BF16 and FP8 e4m3 only
+    bad = qsa.qsa.qsa_cache_t(0x1000, 0x1000, 0x1000, 0x1000, 10, 2, 4, 2, 7)
+    bp = ctypes.byref(bad)
+    assert L.qsa_append_kv(bp, fake, fake, fake, fake, fake, 5, None, None) == -2
+    assert L.qsa_sparse_decode(bp, fake, 1, 16, fake, fake, fake, fake, 16, 0.0625, 16, 4, fake, fake, None, None) == -2
 
 
 def test_binding_rejects_host_tensors():

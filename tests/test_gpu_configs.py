@@ -21,6 +21,8 @@ SAMPLES = {
     "long": [0, 17, 31],
     "quarter": None,            # shortest, longest and two more
     "prefill": [0, 1, 2, 3, 4095, 4096, 6001, 8191],
+    "long-fp8": [0, 17, 31],
+    "quarter-fp8": None,
 }
 
 
@@ -30,7 +32,7 @@ def _need_cuda():
         pytest.skip("needs a CUDA device")
 
 
-@pytest.mark.parametrize("name", list(C.ALL))
+@pytest.mark.parametrize("name", list(C.ALL) + list(C.FP8))
 def test_workload_full_size(name):
     wl = C.get(name)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")

@@ -45,6 +45,7 @@ class Workload:
     spikes: bool = False
     seed: int = 0
     splits_per_query: int = 0  # 0 = balance over the SMs; >0 = about this many KV chunks per query
+    kv_fp8: bool = False       # main K/V cache stored as FP8 e4m3 (the side cache stays BF16)
 
     @property
     def total_lengths(self) -> list[int]:
@@ -66,7 +67,7 @@ class Workload:
                             else [min(self.total_lengths), max(self.total_lengths)]),
                 "new_tokens_per_seq": self.new_tokens, "top_k_blocks": self.k_top,
                 "head_dim": HEAD_DIM, "indexer": f"{IDX_HEADS}x{IDX_DIM}", "page_tokens": PAGE,
-                "page_permutation": self.page_perm}
+                "page_permutation": self.page_perm, "kv_cache": "fp8_e4m3" if self.kv_fp8 else "bf16"}
 
 
 def _decode(name, batch, ctx, hq, hkv, **kw):
@@ -86,6 +87,10 @@ def get(name: str) -> Workload:
     if name == "quarter":
         lens = synth.sequence_lengths(0, 64, 16384, 262144)
         return _decode("decode-b64-ctx16k-262k-h12x1-paged", 64, lens, 12, 1, page_perm=True)
+    if name == "long-fp8":
+        return dataclasses.replace(get("long"), name="decode-b32-ctx131072-h24x2-spiked-fp8kv", kv_fp8=True)
+    if name == "quarter-fp8":
+        return dataclasses.replace(get("quarter"), name="decode-b64-ctx16k-262k-h12x1-paged-fp8kv", kv_fp8=True)
     if name == "prefill":
         return Workload(name="extend-b2-ctx65536+4096-h6x1", batch=2, hq=6, hkv=1,
                         lengths=(65536, 65536), new_tokens=4096)
@@ -93,6 +98,7 @@ def get(name: str) -> Workload:
 
 
 ALL = ("tiny", "batched", "long", "quarter", "prefill")
+FP8 = ("long-fp8", "quarter-fp8")   # the same decode workloads with an FP8 e4m3 main K/V cache
 
 
 def shrink(wl: Workload, lengths, new_tokens=None, k_top=None, name=None, **kw) -> Workload:

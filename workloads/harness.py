@@ -17,7 +17,8 @@ from . import configs as C
 def new_cache(wl: C.Workload, device="cuda", block_table=None) -> qsa.PagedCache:
     bt = C.block_table(wl) if block_table is None else block_table
     return qsa.PagedCache(num_pages=wl.num_pages(), max_seqs=wl.batch, max_pages_per_seq=wl.pages_per_seq(),
-                          num_kv_heads=wl.hkv, block_table=bt, device=device)
+                          num_kv_heads=wl.hkv, block_table=bt, device=device,
+                          kv_dtype=qsa.KV_FP8_E4M3 if wl.kv_fp8 else qsa.KV_BF16)
 
 
 def append_range(cache: qsa.PagedCache, wl: C.Workload, seq: int, start: int, stop: int, dev_status=None,
