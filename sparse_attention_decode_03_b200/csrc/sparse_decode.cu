@@ -153,8 +153,10 @@ __device__ __forceinline__ Seg make_seg(const DecodeArgs& a, int64_t pair, int64
   s.u0 = (int)(max(x0, base) - base);
   s.u1 = (int)(min(x1, base + n_slots) - base);
   s.last_of_pair = s.u1 == (int)n_slots;
+  // the three per-query loads are independent: issued together, one latency
   s.seq = a.q_seq[s.q];
   const int p = a.q_pos[s.q];
+  const int cnt_raw = a.count[s.q];
   s.query_ok = s.seq >= 0 && s.seq < a.max_seqs && p >= 0 && (int64_t)p < (int64_t)a.mpps * kPage;
   if (!s.query_ok) {
     if (report) flag(a.st, (s.seq < 0 || s.seq >= a.max_seqs) ? QSA_DEV_BAD_SEQ : QSA_DEV_BAD_POS);
@@ -164,7 +166,7 @@ __device__ __forceinline__ Seg make_seg(const DecodeArgs& a, int64_t pair, int64
     s.nb = (p + 1) / kRatio;
     s.t = (p + 1) % kRatio;
   }
-  int cnt = s.query_ok ? a.count[s.q] : 0;
+  int cnt = s.query_ok ? cnt_raw : 0;
   const int cap = min(a.K, s.nb);
   if (cnt < 0 || cnt > cap) {
     if (report) flag(a.st, QSA_DEV_BAD_COUNT);
@@ -468,8 +470,8 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
     for (int idx = tid; idx < 16 * 32; idx += kConsumerThreads) {
       const int row = idx >> 5, c = idx & 31;
       uint4 v = make_uint4(0, 0, 0, 0);
-      if (row < G && s.query_ok)
-        v = ldg_nc(a.q + ((size_t)s.q * a.hq + (size_t)s.g * G + row) * kHeadDim + c * 8);
+      if (row < G) v = ldg_nc(a.q + ((size_t)s.q * a.hq + (size_t)s.g * G + row) * kHeadDim + c * 8);
+      if (!s.query_ok) v = make_uint4(0, 0, 0, 0);
       if constexpr (F8) {
         uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll

@@ -17,7 +17,7 @@
 //      loads) and appends the keys >= T0 with their indices to its own
 //      shared-memory list, in index order (ballots and a warp scan);
 //   3. exact select among the candidates: radix passes (12-bit windows from
-//      the candidates' highest differing bit, warp-aggregated atomics) give a
+//      the candidates' highest differing bit, shared-memory atomics) give a
 //      prefix T under a mask with "every key above T, and the first `need`
 //      keys equal to T in index order" = the top K;
 //   4. ordered output: warp totals scanned once, then each warp writes its
@@ -175,13 +175,11 @@ struct TopkSmem {
   uint32_t above;
 };
 
-// Add 1 to hist[bin] for every live lane: one atomic per distinct bin per warp.
+// Add 1 to hist[bin] for every live lane.  Plain shared-memory atomics: the
+// hardware serialises lanes that hit the same bin, which costs less than
+// aggregating them with __match_any_sync first (measured on B200).
 __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool live) {
-  const uint32_t act = __ballot_sync(0xffffffffu, live);
-  if (live) {
-    const uint32_t peers = __match_any_sync(act, bin);
-    if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
-  }
+  if (live) atomicAdd(&hist[bin], 1u);
 }
 
 // Block-wide min and max of one value per thread.
