@@ -298,7 +298,13 @@ def run_native(args, rank, ws, local):
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     st = torch.zeros(1, dtype=torch.int32, device=dev)
     cache = H.build_cache(wl, dev_status=st)
-    inp = H.step_inputs(wl)
+    # the step's inputs live in one staged buffer (one host-to-device copy per step in the e2e leg)
+    io = qsa.StepIO(wl.batch * wl.new_tokens, wl.nq, wl.hq, wl.hkv, dev)
+    for k, t in H.step_inputs(wl, device="cpu").items():
+        io.host[k].copy_(t)
+    io.upload()
+    torch.cuda.synchronize()
+    inp = io.dev
     dec = qsa.Decoder(cache, wl.hq, wl.nq, k=wl.k_top, scale=wl.scale, target_ctas=sms,
                       chunk_units=H.chunk_units_for(wl))
     dec.dev_status = st
@@ -401,23 +407,19 @@ def run_native(args, rank, ws, local):
     if status:
         raise RuntimeError(f"device status after the kernel timing: {qsa.dev_status_names(status)}")
 
-    # ---- e2e: pinned host buffers, H2D of the step's inputs + the step (graph) + D2H of out/lse
-    keys = ["k_new", "v_new", "kidx_new", "seq_id", "pos", "q", "q_idx", "w", "q_seq", "q_pos"]
-    host = {k: inp[k].cpu().pin_memory() for k in keys}
-    out_h = torch.empty(dec.out[:wl.nq].shape, dtype=dec.out.dtype).pin_memory()
-    lse_h = torch.empty(dec.lse[:wl.nq].shape, dtype=dec.lse.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+    # ---- e2e: the step's inputs from pinned host memory (one copy of the staged
+    # buffer) + the step (graph) + out/lse back to pinned host memory
+    out_host = dec.host_outputs()
+    h2d = io.nbytes
+    d2h = 0
     e2e_ms = []
     for i in range(args.steps + 2):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
             e0.record(stream)
-            for k in keys:
-                inp[k].copy_(host[k], non_blocking=True)
+            io.upload(stream)
             graph.replay()
-            out_h.copy_(dec.out[:wl.nq], non_blocking=True)
-            lse_h.copy_(dec.lse[:wl.nq], non_blocking=True)
+            d2h = dec.download(out_host, wl.nq, stream)
             e1.record(stream)
         e1.synchronize()
         if i >= 2:

@@ -330,8 +330,11 @@ class Decoder:
         self.count = torch.empty((max_nq,), dtype=torch.int32, device=dev)
         self.part_o = torch.empty((max_nq, self.max_splits, hq, HEAD_DIM), dtype=torch.float32, device=dev)
         self.part_lse = torch.empty((max_nq, self.max_splits, hq), dtype=torch.float32, device=dev)
-        self.out = torch.empty((max_nq, hq, HEAD_DIM), dtype=torch.bfloat16, device=dev)
-        self.lse = torch.empty((max_nq, hq), dtype=torch.float32, device=dev)
+        # out and lse share one allocation, so a full batch reads back in one copy
+        out_bytes = max_nq * hq * HEAD_DIM * 2
+        self._out_arena = torch.empty(_align(out_bytes) + max_nq * hq * 4, dtype=torch.uint8, device=dev)
+        self.out = self._out_arena[:out_bytes].view(torch.bfloat16).view(max_nq, hq, HEAD_DIM)
+        self.lse = self._out_arena[_align(out_bytes):].view(torch.float32).view(max_nq, hq)
         self.dev_status = torch.zeros((1,), dtype=torch.int32, device=dev)
 
     def bind(self, q, q_idx, w, q_seq, q_pos, stream=None) -> list:
@@ -362,6 +365,27 @@ class Decoder:
             BoundCall("qsa_combine", (_ptr(po), _ptr(pl), nq, self.max_splits, hq, _ptr(out), _ptr(lse), sp), keep),
         ]
 
+    def host_outputs(self):
+        """Pinned host buffers laid out like the device outputs: (arena, out, lse)."""
+        arena = torch.empty(self._out_arena.shape, dtype=torch.uint8).pin_memory()
+        out = arena[:self.out.numel() * 2].view(torch.bfloat16).view(self.out.shape)
+        lse = arena[self._out_arena.numel() - self.lse.numel() * 4:].view(torch.float32).view(self.lse.shape)
+        return arena, out, lse
+
+    def download(self, host, nq: int, stream=None) -> int:
+        """Enqueue the device-to-host copy of out[:nq] and lse[:nq] into `host`
+        (from host_outputs()): one copy for a full batch, two otherwise.
+        Returns the bytes copied."""
+        arena, out, lse = host
+        s = stream or torch.cuda.current_stream()
+        with torch.cuda.stream(s):
+            if nq == self.max_nq:
+                arena.copy_(self._out_arena, non_blocking=True)
+                return arena.numel()
+            out[:nq].copy_(self.out[:nq], non_blocking=True)
+            lse[:nq].copy_(self.lse[:nq], non_blocking=True)
+        return out[:nq].numel() * 2 + lse[:nq].numel() * 4
+
     def run(self, q, q_idx, w, q_seq, q_pos, stream=None):
         nq = int(q_seq.shape[0])
         assert nq <= self.max_nq
@@ -373,6 +397,43 @@ class Decoder:
                           self.max_splits, po, pl, self.dev_status, stream)
         qsa_combine(po, pl, self.out[:nq], self.lse[:nq], stream)
         return self.out[:nq], self.lse[:nq]
+
+
+def _align(n: int, a: int = 256) -> int:
+    return (n + a - 1) // a * a
+
+
+class StepIO:
+    """The inputs of one step (the appended tokens and the queries) staged in one
+    pinned host buffer and one device buffer, 256-byte aligned fields, so that
+    sending a step's inputs is a single host-to-device copy.  `host[name]` and
+    `dev[name]` are views of the same field; bind the step to the `dev` views,
+    fill the `host` views, then upload()."""
+
+    def __init__(self, n_new: int, nq: int, hq: int, hkv: int, device="cuda"):
+        fields = [("k_new", torch.bfloat16, (n_new, hkv, HEAD_DIM)), ("v_new", torch.bfloat16, (n_new, hkv, HEAD_DIM)),
+                  ("kidx_new", torch.bfloat16, (n_new, IDX_DIM)), ("seq_id", torch.int32, (n_new,)),
+                  ("pos", torch.int32, (n_new,)), ("q", torch.bfloat16, (nq, hq, HEAD_DIM)),
+                  ("q_idx", torch.bfloat16, (nq, IDX_HEADS, IDX_DIM)), ("w", torch.float32, (nq, IDX_HEADS)),
+                  ("q_seq", torch.int32, (nq,)), ("q_pos", torch.int32, (nq,))]
+        off, spans = 0, []
+        for name, dt, shape in fields:
+            nbytes = torch.Size(shape).numel() * torch.empty((), dtype=dt).element_size()
+            spans.append((name, dt, shape, off, nbytes))
+            off = _align(off + nbytes)
+        self.nbytes = off
+        self.host_buf = torch.empty(off, dtype=torch.uint8).pin_memory()
+        self.dev_buf = torch.empty(off, dtype=torch.uint8, device=device)
+        self.host, self.dev = {}, {}
+        for name, dt, shape, o, nb in spans:
+            self.host[name] = self.host_buf[o:o + nb].view(dt).view(shape)
+            self.dev[name] = self.dev_buf[o:o + nb].view(dt).view(shape)
+
+    def upload(self, stream=None):
+        """Enqueue the single host-to-device copy of every field."""
+        s = stream or torch.cuda.current_stream()
+        with torch.cuda.stream(s):
+            self.dev_buf.copy_(self.host_buf, non_blocking=True)
 
 
 class StepGraph:

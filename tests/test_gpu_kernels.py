@@ -453,3 +453,48 @@ def test_split_pipeline_stress_no_expired_waits():
     assert int(dec.dev_status.item()) == 0, qsa.dev_status_names(int(dec.dev_status.item()))
     assert torch.equal(dec.out.view(torch.int16), ref_o.view(torch.int16))
     assert torch.equal(dec.part_lse, ref_l)
+
+
+def test_step_io_staging_and_readback():
+    """The staged step inputs (one host-to-device copy) drive the same step as
+    separately allocated inputs, bit for bit, and the output read-back (one
+    copy for a full batch, two for a partial one) returns the device values."""
+    wl = C.shrink(C.get("long"), [3000, 2050, 777], k_top=64)
+    st = _status()
+    cache = H.build_cache(wl, dev_status=st)
+    ref_in = H.step_inputs(wl)
+    io = qsa.StepIO(wl.batch * wl.new_tokens, wl.nq, wl.hq, wl.hkv)
+    for k, t in H.step_inputs(wl, device="cpu").items():
+        io.host[k].copy_(t)
+    io.upload()
+    torch.cuda.synchronize()
+    for k, t in ref_in.items():
+        assert torch.equal(io.dev[k], t), k
+    saved = cache.kc_partial.clone()
+    outs = []
+    for inp in (ref_in, io.dev):
+        cache.kc_partial.copy_(saved)
+        qsa.qsa_append_kv(cache, inp["k_new"], inp["v_new"], inp["kidx_new"], inp["seq_id"], inp["pos"], st)
+        dec = qsa.Decoder(cache, wl.hq, wl.nq, k=64)
+        dec.dev_status = st
+        dec.run(inp["q"], inp["q_idx"], inp["w"], inp["q_seq"], inp["q_pos"])
+        host = dec.host_outputs()
+        nbytes = dec.download(host, wl.nq)
+        torch.cuda.synchronize()
+        assert nbytes == host[0].numel()
+        assert torch.equal(host[1].view(torch.int16), dec.out.cpu().view(torch.int16))
+        assert torch.equal(host[2], dec.lse.cpu())
+        outs.append(dec.out.clone())
+    assert int(st.item()) == 0
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    # a partial batch reads back its rows only
+    dec2 = qsa.Decoder(cache, wl.hq, wl.nq + 5, k=64)
+    dec2.dev_status = st
+    dec2.run(io.dev["q"], io.dev["q_idx"], io.dev["w"], io.dev["q_seq"], io.dev["q_pos"])
+    host = dec2.host_outputs()
+    host[1].zero_()
+    nbytes = dec2.download(host, wl.nq)
+    torch.cuda.synchronize()
+    assert nbytes == wl.nq * wl.hq * 256 * 2 + wl.nq * wl.hq * 4
+    assert torch.equal(host[1][:wl.nq].view(torch.int16), dec2.out[:wl.nq].cpu().view(torch.int16))
+    assert torch.all(host[1][wl.nq:] == 0)
