@@ -47,7 +47,10 @@ Readings where the pages are silent (each is listed in the design notes):
     lse_s = -inf gives o = 0 exactly and lse = -inf;
   * the FP8 main K/V cache stores e4m3(K) and e4m3(V) of the BF16 rows (round
     to nearest even, saturated, no scale); attention runs on those values and
-    the indexer side cache stays BF16.
+    the indexer side cache stays BF16;
+  * DCP: page P = position // 64 of a sequence lives on rank (P // I) % N; a
+    rank attends to the attended tokens it holds; the ranks' (o, lse) are
+    merged by the same log-sum-exp combine as the splits.
 
 Every function below is pinned by tests in ``tests/test_oracle_pins.py``
 against closed forms, library routines or brute force; no function is
@@ -301,3 +304,35 @@ def combine(part_o, part_lse):
         lse[h] = m + np.log(L)
         o[h] = (wts[:, None] * po[live, h]).sum(axis=0) / L
     return o, lse
+
+
+# ----------------------------------------------------------------------------
+# decode context parallelism (DCP)
+#
+# [DCP] "Qwen 4 QSA krijgt decode-contextparallellisme ...", section "Wat de
+# pull request daadwerkelijk verandert": the main KV is split by context over
+# the ranks, each rank reads its own slice, the selection is the same on every
+# rank (the selector is replicated), and the ranks' partial attention results
+# are combined.  The shard rule is a reading (the pages give none): logical
+# page P = position // 64 of a sequence lives on rank (P // I) % N.
+
+PAGE_TOKENS = 64
+
+
+def dcp_owner(position, nranks: int, interleave_pages: int = 1):
+    """Rank holding the K/V of a token position (array or scalar)."""
+    page = np.asarray(position, dtype=np.int64) // PAGE_TOKENS
+    return (page // interleave_pages) % nranks
+
+
+def dcp_rank_partial(q_heads, sel, p: int, kv_rows, scale: float, nranks: int, rank: int,
+                     interleave_pages: int = 1):
+    """One rank's share of a query: attention of every Q head over the attended
+    tokens (selected blocks and trailing tokens) that the rank holds.
+    Returns (o [Hq][256], lse [Hq]); a rank holding none of them gives o = 0,
+    lse = -inf."""
+    pos = token_positions(sel, p)
+    mine = pos[dcp_owner(pos, nranks, interleave_pages) == rank]
+    K, V = kv_rows(mine)
+    return attend_gqa(q_heads, K, V, scale) if mine.shape[0] else (
+        np.zeros((np.asarray(q_heads).shape[0], HEAD_DIM)), np.full(np.asarray(q_heads).shape[0], -np.inf))

@@ -319,3 +319,38 @@ def test_fully_masked_row_is_zero():
     r = O.decode_query(q, qi, w, 3, kidx, lambda pos: (K[pos], V[pos]), k=0, scale=1 / 16)  # nb=1, t=0, K=0
     assert r["positions"].shape == (0,)
     assert np.all(r["o"] == 0) and np.all(np.isneginf(r["lse"]))
+
+
+# ---------------------------------------------------------------- DCP (decode context parallelism)
+
+def test_dcp_owner_follows_the_page_rule():
+    pos = np.array([0, 63, 64, 127, 128, 191, 192, 255, 256, 320])
+    # round robin by page over 2 ranks, and pairs of pages over 2 ranks
+    assert O.dcp_owner(pos, 2, 1).tolist() == [0, 0, 1, 1, 0, 0, 1, 1, 0, 1]
+    assert O.dcp_owner(pos, 2, 2).tolist() == [0, 0, 0, 0, 1, 1, 1, 1, 0, 0]
+    assert O.dcp_owner(pos, 3, 1).tolist() == [0, 0, 1, 1, 2, 2, 0, 0, 1, 2]
+    assert np.all(O.dcp_owner(pos, 1, 1) == 0)
+
+
+@pytest.mark.parametrize("nranks,interleave", [(1, 1), (2, 1), (3, 1), (4, 1), (2, 2), (3, 2)])
+def test_dcp_rank_partials_merge_to_the_unsharded_result(nranks, interleave):
+    """The ranks' shares partition the attended tokens, so their log-sum-exp
+    merge is the unsharded attention (fp64 rounding only), including ranks that
+    hold nothing of a query and tails on any rank."""
+    hq, hkv, k = 12, 2, 24
+    L = 64 * 7 + 13
+    K, V, kidx, q, qi, w = _toy(L, hq, hkv, seed=nranks * 10 + interleave)
+    rows = lambda pos: (K[pos], V[pos])
+    for p in (L - 1, 64 * 3 + 1, 64 * 5 - 1, 70, 2):
+        r = O.decode_query(q, qi, w, p, kidx, rows, k=k, scale=1 / 16)
+        parts = [O.dcp_rank_partial(q, r["sel"], p, rows, 1 / 16, nranks, rank, interleave) for rank in range(nranks)]
+        po = np.stack([x[0] for x in parts])
+        pl = np.stack([x[1] for x in parts])
+        n_tok = sum(int(np.sum(O.dcp_owner(r["positions"], nranks, interleave) == rank)) for rank in range(nranks))
+        assert n_tok == len(r["positions"])
+        o, lse = O.combine(po, pl)
+        assert np.allclose(o, r["o"], rtol=1e-12, atol=1e-12)
+        assert np.allclose(lse, r["lse"], rtol=1e-12)
+        for rank in range(nranks):   # a rank without tokens contributes o = 0, lse = -inf
+            if not np.any(O.dcp_owner(r["positions"], nranks, interleave) == rank):
+                assert np.all(parts[rank][0] == 0) and np.all(np.isneginf(parts[rank][1]))
