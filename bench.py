@@ -51,6 +51,9 @@ def parse_args():
     ap.add_argument("--context", type=int, default=0, help="override every context length (profiling a small case)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time budget for the CPU baseline")
+    ap.add_argument("--dcp", type=int, default=0,
+                    help="decode context parallelism over this many ranks: time rank 0's share of a step on one GPU")
+    ap.add_argument("--dcp-interleave", type=int, default=1, help="DCP shard interleave, in 64-token pages")
     return ap.parse_args()
 
 
@@ -431,7 +434,7 @@ def run_native(args, rank, ws, local):
         raise RuntimeError(f"device status after the e2e steps: {qsa.dev_status_names(status)}")
     e2e_total = max_over_ranks(sum(e2e_ms), ws)
     e2e_value = ws * wl.nq * len(e2e_ms) / (e2e_total / 1000.0)
-    launches_per_step = 6 + (1 if dec.scores_ld > 65536 else 0)
+    launches_per_step = 6  # append scatter + append partial + scores + top-K + attention + combine
 
     # ---- roofline of the dominant kernel
     count = dec.count[:wl.nq].cpu().numpy()
@@ -479,12 +482,151 @@ def run_native(args, rank, ws, local):
         print(json.dumps(line), flush=True)
 
 
+def run_dcp(args, rank, ws, local):
+    """Rank 0 of a DCP group of args.dcp ranks, on one GPU: its replicated
+    selector and its K/V shard, and its share of every step (append, scores,
+    top-K, localisation, attention over its blocks, merge of its splits, and
+    the merge over the ranks).  The all-gather of the ranks' (o, lse) between
+    the attention and the final merge is not timed (one GPU: no peer)."""
+    import sparse_attention_decode_03_b200 as qsa
+    from workloads import harness as H
+
+    if ws != 1:
+        raise SystemExit("--dcp times one rank's share on one GPU; run it without torchrun")
+    R, I = args.dcp, args.dcp_interleave
+    wl = C.get(args.workload)
+    if args.batch:
+        wl = C.shrink(wl, list(wl.lengths[:args.batch]), name=f"{wl.name}-first{args.batch}")
+    dev = torch.device("cuda", local)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    sh = qsa.DCPShard(R, 0, I)
+    pages = [-(-L // 64) for L in wl.total_lengths]
+    selector = qsa.PagedCache(wl.num_pages(), wl.batch, wl.pages_per_seq(), wl.hkv, block_table=C.block_table(wl),
+                              device=dev, with_kv=False)
+    bt, used = sh.shard_block_table(pages)
+    shard = qsa.PagedCache(max(1, used), wl.batch, bt.shape[1], wl.hkv, block_table=bt, device=dev, with_kc=False,
+                           kv_dtype=qsa.KV_FP8_E4M3 if wl.kv_fp8 else qsa.KV_BF16)
+    rk = qsa.DCPRank(selector, shard, wl.hq, wl.nq, R, 0, I, k=wl.k_top, scale=wl.scale)
+    rk.dev_status = st
+    for b, L in enumerate(wl.lengths):
+        for a0 in range(0, L, 32768):
+            a1 = min(L, a0 + 32768)
+            pos = torch.arange(a0, a1, device=dev)
+            rk.append(C.k_rows(wl, b, pos, dev), C.v_rows(wl, b, pos, dev), C.kidx_rows(wl, b, pos, dev),
+                      torch.full((a1 - a0,), b, dtype=torch.int32, device=dev), pos.to(torch.int32))
+    inp = H.step_inputs(wl, device=dev)
+    saved = selector.kc_partial.clone()
+    stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    flush_read = torch.ones(64 << 20, dtype=torch.int32, device=dev)
+    flush_sink = torch.zeros((), dtype=torch.int64, device=dev)
+
+    def flush_l2():
+        flush.zero_()
+        flush_sink.copy_(flush_read.sum())
+
+    def between():
+        with torch.cuda.stream(stream):
+            selector.kc_partial.copy_(saved)
+            flush_l2()
+
+    def step():
+        rk.append(inp["k_new"], inp["v_new"], inp["kidx_new"], inp["seq_id"], inp["pos"], stream)
+        rk.attend(inp["q"], inp["q_idx"], inp["w"], inp["q_seq"], inp["q_pos"], stream)
+        rk.merge(wl.nq, stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+            for j in range(R):               # the exchange, emulated once outside the timed steps
+                rk.o_all[j].copy_(rk.o_rank)
+                rk.lse_all[j].copy_(rk.lse_rank)
+            between()
+    torch.cuda.synchronize()
+    if int(st.item()):
+        raise RuntimeError(f"device status {qsa.dev_status_names(int(st.item()))}")
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        step()
+    for _ in range(3):
+        with torch.cuda.stream(stream):
+            g.replay()
+        between()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            with torch.cuda.stream(stream):
+                evs[i][0].record(stream)
+                g.replay()
+                evs[i][1].record(stream)
+            between()
+        torch.cuda.synchronize()
+    if int(st.item()):
+        raise RuntimeError(f"device status after the timed steps: {qsa.dev_status_names(int(st.item()))}")
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    mean_ms = statistics.mean(step_ms)
+    # the shard attention kernel alone, cold L2 (graph of 8 x (flush, kernel) minus 8 x flush)
+    nq = wl.nq
+    decode_call = lambda: qsa.qsa_sparse_decode(
+        shard, inp["q"], inp["q_seq"], rk.q_pos_local[:nq], rk.sel_local[:nq], rk.count_local[:nq], rk.k, rk.scale,
+        rk.chunk_units, rk.max_splits, rk.part_o[:nq], rk.part_lse[:nq], st, stream)
+
+    def gtime(fns):
+        gg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gg, stream=stream):
+            for _ in range(8):
+                for f in fns:
+                    f()
+        best = 1e9
+        for _ in range(6):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                gg.replay()
+                e1.record(stream)
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        return best
+    dec_ms = max(gtime([flush_l2, decode_call]) - gtime([flush_l2]), 1e-6) / 8
+    torch.cuda.synchronize()
+    tok_kv = wl.hkv * 256 * 2 * (1 if wl.kv_fp8 else 2)
+    cl = rk.count_local[:nq].cpu().numpy().astype(np.int64)
+    ql = rk.q_pos_local[:nq].cpu().numpy().astype(np.int64)
+    qp = inp["q_pos"].cpu().numpy().astype(np.int64)
+    tail_here = ((ql + 1) % 4 == (qp + 1) % 4) & ((qp + 1) % 4 > 0)
+    sel_tokens = int((4 * cl).sum() + ((qp + 1) % 4)[tail_here].sum())
+    dec_bytes = sel_tokens * tok_kv + nq * wl.hq * 256 * 2
+    peak, peak_kind = measured_peaks()
+    achieved = dec_bytes / (dec_ms / 1000.0) / 1e9
+    line = {
+        "metric": METRIC, "value": nq / (mean_ms / 1000.0), "unit": "queries/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": mean_ms, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "e4m3 kv + bf16" if wl.kv_fp8 else "bf16", "data": "synthetic",
+        "config": {**wl.describe(), "parallelism": f"dcp{R} (interleave {I} pages): rank 0 of {R} on one GPU, "
+                   "its own K/V shard and a replicated selector; the all-gather of the ranks' (o, lse) is not timed",
+                   "step": "append (side cache + shard) + index_scores + topk + localize + sparse_decode (shard) + "
+                           "merge of the rank's splits + merge over the ranks, one CUDA graph",
+                   "l2": "flushed between timed steps"},
+        "roofline": {"kernel": "sparse_decode (rank 0 shard)", "bound": "hbm", "achieved": round(achieved, 1),
+                     "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "alg_bytes_per_launch": dec_bytes, "peak_kind": f"{peak_kind} (hbm_gbs)",
+                     "ms": round(dec_ms, 5)},
+        "rank0_selected_blocks": int(cl.sum()), "all_selected_blocks": int(rk.count[:nq].sum()),
+        "gpu_launches": 10 * args.steps,  # 2 + 1 + 1 appends and localisation, scores, top-K, localisation, attention, 2 merges
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     rank, ws, local = dist_init()
     try:
         if args.impl == "reference":
             run_reference(args, rank, ws)
+        elif args.dcp > 1:
+            run_dcp(args, rank, ws, local)
         else:
             run_native(args, rank, ws, local)
     finally:

@@ -104,6 +104,11 @@ typedef enum {
  *               sparse attention gathers.  The side cache stays BF16.
  * All buffers are caller-owned device memory; the library writes kv/kc pages
  * and kc_partial only in qsa_append_kv.
+ * A group may leave out one part: kv_pages NULL (a selector-only group, e.g.
+ * the replicated side cache of a DCP rank) or kc_pages and kc_partial NULL (a
+ * main-K/V-only group, e.g. a DCP rank's K/V shard).  qsa_append_kv then
+ * writes only the part that is there; qsa_index_scores needs kc_pages and
+ * qsa_sparse_decode needs kv_pages.
  */
 #define QSA_KV_BF16 0
 #define QSA_KV_FP8_E4M3 1
@@ -124,7 +129,7 @@ QSA_API const char* qsa_status_string(int status);
 
 /* ABI version of this header (bumped on any signature change). */
 QSA_API int qsa_abi_version(void);
-#define QSA_ABI_VERSION 3
+#define QSA_ABI_VERSION 4
 
 /*
  * qsa_append_kv -- write n new tokens into the cache group.
@@ -228,6 +233,64 @@ QSA_API int qsa_sparse_decode(const qsa_cache_t* cache, const void* q, int32_t n
  */
 QSA_API int qsa_combine(const float* part_o, const float* part_lse, int32_t nq, int32_t max_splits, int32_t hq,
                 void* out, float* lse, void* stream);
+
+/*
+ * qsa_combine_strided -- the same merge over nsplits splits laid out with
+ * explicit element strides: split s of (query q, head h) is
+ *   part_o[q * o_q_stride + s * o_split_stride + h * 256 + d],
+ *   part_lse[q * lse_q_stride + s * lse_split_stride + h];
+ * qsa_combine is the case o_split_stride = hq*256, o_q_stride = S*hq*256,
+ * lse_split_stride = hq, lse_q_stride = S*hq.  With out_dtype QSA_OUT_F32 the
+ * merged rows are written as fp32 (16-byte aligned out), so a merged result can
+ * itself be one split of a later merge: a DCP rank merges its own splits, the
+ * ranks' results are gathered rank-major ([rank][q][h][256], o_split_stride =
+ * nq*hq*256) and merged again ([DCP]: split results combined across ranks).
+ * o strides must be multiples of 4 elements.
+ */
+#define QSA_OUT_BF16 0
+#define QSA_OUT_F32 1
+QSA_API int qsa_combine_strided(const float* part_o, const float* part_lse, int32_t nq, int32_t nsplits, int32_t hq,
+                        int64_t o_q_stride, int64_t o_split_stride, int64_t lse_q_stride,
+                        int64_t lse_split_stride, void* out, int32_t out_dtype, float* lse, void* stream);
+
+/*
+ * Decode context parallelism ([DCP] "Qwen 4 QSA krijgt
+ * decode-contextparallellisme ...", section "Wat de pull request daadwerkelijk
+ * verandert"): the main K/V of each sequence is sharded by context over
+ * nranks ranks while the selector (side cache, scores, top-K) is replicated;
+ * each rank attends to the selected blocks it holds and the ranks' results are
+ * merged by log-sum-exp.  Shard rule (a reading; the pages do not give one):
+ * logical page P (64 tokens) of a sequence lives on rank (P / I) % nranks at
+ * local page (P / (I*nranks)) * I + P % I, I = interleave_pages >= 1.  A
+ * rank's K/V shard is a main-K/V-only cache group whose block table maps local
+ * pages.
+ *
+ * qsa_dcp_localize_tokens -- the rank's view of a batch of appended tokens:
+ *   seq_id_local[i] = seq_id[i] if the rank holds the token's page, else -1
+ *   pos_local[i]    = its local position (local page * 64 + pos % 64), else 0
+ * so qsa_append_kv on the shard writes exactly the rank's tokens.
+ */
+QSA_API int qsa_dcp_localize_tokens(const int32_t* seq_id, const int32_t* pos, int32_t n, int32_t nranks,
+                            int32_t rank, int32_t interleave_pages, int32_t* seq_id_local, int32_t* pos_local,
+                            void* stream);
+
+/*
+ * qsa_dcp_localize_selection -- the localisation step ([DCP] "the QSA
+ * localization kernel"): for each query, the entries of the global selection
+ * (sel/count from qsa_topk_blocks) that the rank holds, in order, as local block
+ * indices (local page * 16 + j % 16), -1 padded to k; their number; and a
+ * local position q_pos_local whose nb and tail make qsa_sparse_decode on the
+ * shard attend to exactly those blocks, plus the trailing tokens when the rank
+ * holds the page they are in (a rank holding nothing of a query gets count 0
+ * and q_pos_local 3).  A query with q_pos < 0 is passed through with count 0.
+ * Out-of-range entries set QSA_DEV_BAD_SEL and are dropped; a count outside
+ * [0, min(k, nb)] sets QSA_DEV_BAD_COUNT and is clamped.
+ *   sel, sel_local int32 [nq][k]; count, count_local, q_pos, q_pos_local int32 [nq]
+ */
+QSA_API int qsa_dcp_localize_selection(const int32_t* sel, const int32_t* count, const int32_t* q_pos, int32_t nq,
+                               int32_t k, int32_t nranks, int32_t rank, int32_t interleave_pages,
+                               int32_t* sel_local, int32_t* count_local, int32_t* q_pos_local,
+                               int32_t* dev_status, void* stream);
 
 /*
  * qsa_sparse_attention_noalloc -- qsa_sparse_decode then qsa_combine in one

@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(kWarps * 32) append_scatter_kernel(AppendArgs 
   }
   const int slot = p % kPage;
   const int hkv = a.c.num_kv_heads;
-  for (int h = 0; h < hkv; ++h) {
+  for (int h = 0; a.c.kv_pages && h < hkv; ++h) {  // no main K/V in a selector-only group
     // [page][h][micro-block][K rows | V rows][256] elements
     const size_t blk = (((size_t)page * hkv + h) * kBlocksPerPage + slot / kRatio) * (2 * kRatio * kHeadDim);
     const size_t dst = blk + (size_t)(slot % kRatio) * kHeadDim + lane * 8;
@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(kWarps * 32) append_scatter_kernel(AppendArgs 
       *reinterpret_cast<uint4*>(kv + dst + kRatio * kHeadDim) = vv8;
     }
   }
-  if ((p & 3) == 3) {  // this token closes micro-block p / 4
+  if (a.c.kc_pages && (p & 3) == 3) {  // this token closes micro-block p / 4
     const int m = run_before(a, tok, seq, p, 3);
     const float4 acc = block_sum(a, tok, seq, m, m < 3, lane);
     __nv_bfloat16* kc = static_cast<__nv_bfloat16*>(a.c.kc_pages) +
@@ -166,12 +166,16 @@ extern "C" int qsa_append_kv(const qsa_cache_t* cache, const void* k_new, const 
   if (!cache || n < 0) return QSA_ERR_INVALID_ARG;
   if (n == 0) return QSA_OK;
   const qsa_cache_t& c = *cache;
-  if (!c.kv_pages || !c.kc_pages || !c.kc_partial || !c.block_table) return QSA_ERR_INVALID_ARG;
-  if (!k_new || !v_new || !kidx_new || !seq_id || !pos) return QSA_ERR_INVALID_ARG;
+  // a group may hold only the main K/V (kc_pages NULL) or only the side cache (kv_pages NULL)
+  const bool has_kv = c.kv_pages != nullptr, has_kc = c.kc_pages != nullptr;
+  if ((!has_kv && !has_kc) || !c.block_table || !seq_id || !pos) return QSA_ERR_INVALID_ARG;
+  if (has_kv && (!k_new || !v_new)) return QSA_ERR_INVALID_ARG;
+  if (has_kc && (!c.kc_partial || !kidx_new)) return QSA_ERR_INVALID_ARG;
   if (c.num_pages < 1 || c.max_seqs < 1 || c.max_pages_per_seq < 1 || c.num_kv_heads < 1) return QSA_ERR_INVALID_ARG;
   if (c.kv_dtype != QSA_KV_BF16 && c.kv_dtype != QSA_KV_FP8_E4M3) return QSA_ERR_UNSUPPORTED;
-  if (!aligned16(c.kv_pages) || !aligned16(c.kc_partial) || !aligned16(k_new) ||
-      !aligned16(v_new) || (reinterpret_cast<uintptr_t>(c.kc_pages) & 7u) || (reinterpret_cast<uintptr_t>(kidx_new) & 7u))
+  if (has_kv && (!aligned16(c.kv_pages) || !aligned16(k_new) || !aligned16(v_new))) return QSA_ERR_INVALID_ARG;
+  if (has_kc && (!aligned16(c.kc_partial) || (reinterpret_cast<uintptr_t>(c.kc_pages) & 7u) ||
+                 (reinterpret_cast<uintptr_t>(kidx_new) & 7u)))
     return QSA_ERR_INVALID_ARG;
   AppendArgs a{c,
                static_cast<const __nv_bfloat16*>(k_new),
@@ -184,6 +188,6 @@ extern "C" int qsa_append_kv(const qsa_cache_t* cache, const void* k_new, const 
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   const unsigned grid = (unsigned)((n + kWarps - 1) / kWarps);
   int rc = qsa_host::launch(append_scatter_kernel, dim3(grid), dim3(kWarps * 32), 0, s, a);
-  if (rc != QSA_OK) return rc;
+  if (rc != QSA_OK || !has_kc) return rc;
   return qsa_host::launch(append_partial_kernel, dim3(grid), dim3(kWarps * 32), 0, s, a);
 }

@@ -14,60 +14,91 @@ using namespace qsa;
 
 constexpr int kThreads = kHeadDim / 4;  // 64: four output dims per thread
 
+struct CombineArgs {
+  const float* part_o;
+  const float* part_lse;
+  int S, hq;
+  int64_t o_q, o_s;  // element strides of part_o between queries / splits (heads: 256)
+  int64_t l_q, l_s;  // element strides of part_lse between queries / splits (heads: 1)
+  void* out;         // bf16 or fp32 [nq][hq][256]
+  float* lse;
+};
+
 // One CTA per (query, head).  Each thread recomputes the S split weights (S
 // lse values, broadcast from L1) and accumulates its 4 dims over the splits
 // with independent 16-byte loads.
-__global__ void __launch_bounds__(kThreads) combine_kernel(const float* __restrict__ part_o,
-                                                           const float* __restrict__ part_lse, int S, int hq,
-                                                           __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+template <bool F32Out>
+__global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
   pdl_launch_dependents();
   pdl_wait_previous();
   const int qh = blockIdx.x;
-  const int q = qh / hq, h = qh % hq;
+  const int q = qh / a.hq, h = qh % a.hq;
   const int tid = threadIdx.x;
-  const float* pl = part_lse + (size_t)q * S * hq + h;
+  const float* pl = a.part_lse + q * a.l_q + h;
   float M = -INFINITY;
-  for (int s = 0; s < S; ++s) M = fmaxf(M, pl[(size_t)s * hq]);
-  uint2* dst = reinterpret_cast<uint2*>(out + (size_t)qh * kHeadDim) + tid;
-  if (M == -INFINITY) {  // every split empty: zero output, lse = -inf
-    *dst = make_uint2(0u, 0u);
-    if (tid == 0) lse[qh] = -INFINITY;
-    return;
-  }
-  float L = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  const float4* po = reinterpret_cast<const float4*>(part_o + ((size_t)q * S * hq + h) * kHeadDim) + tid;
-  const size_t split_stride = (size_t)hq * kHeadDim / 4;
+  for (int s = 0; s < a.S; ++s) M = fmaxf(M, pl[s * a.l_s]);
+  float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+  float lse_v = -INFINITY;
+  if (M != -INFINITY) {  // else every split is empty: zero output, lse = -inf
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float* po = a.part_o + q * a.o_q + (int64_t)h * kHeadDim + 4 * tid;
 #pragma unroll 4
-  for (int s = 0; s < S; ++s) {
-    const float v = pl[(size_t)s * hq];
-    if (v == -INFINITY) continue;
-    const float e = expf(v - M);
-    const float4 x = po[s * split_stride];
-    L += e;
-    acc.x += e * x.x;
-    acc.y += e * x.y;
-    acc.z += e * x.z;
-    acc.w += e * x.w;
+    for (int s = 0; s < a.S; ++s) {
+      const float v = pl[s * a.l_s];
+      if (v == -INFINITY) continue;
+      const float e = expf(v - M);
+      const float4 x = *reinterpret_cast<const float4*>(po + s * a.o_s);
+      L += e;
+      acc.x += e * x.x;
+      acc.y += e * x.y;
+      acc.z += e * x.z;
+      acc.w += e * x.w;
+    }
+    const float inv = 1.f / L;
+    res = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    lse_v = M + logf(L);
   }
-  const float inv = 1.f / L;
-  uint2 o;
-  o.x = pack_bf16(acc.x * inv, acc.y * inv);
-  o.y = pack_bf16(acc.z * inv, acc.w * inv);
-  *dst = o;
-  if (tid == 0) lse[qh] = M + logf(L);
+  if constexpr (F32Out) {
+    reinterpret_cast<float4*>(static_cast<float*>(a.out) + (size_t)qh * kHeadDim)[tid] = res;
+  } else {
+    uint2 o;
+    o.x = pack_bf16(res.x, res.y);
+    o.y = pack_bf16(res.z, res.w);
+    reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + (size_t)qh * kHeadDim)[tid] = o;
+  }
+  if (tid == 0) a.lse[qh] = lse_v;
 }
 
 }  // namespace
 
+extern "C" int qsa_combine_strided(const float* part_o, const float* part_lse, int32_t nq, int32_t nsplits,
+                                   int32_t hq, int64_t o_q_stride, int64_t o_split_stride, int64_t lse_q_stride,
+                                   int64_t lse_split_stride, void* out, int32_t out_dtype, float* lse, void* stream) {
+  if (nq < 0 || nsplits < 1 || hq < 1) return QSA_ERR_INVALID_ARG;
+  if (out_dtype != QSA_OUT_BF16 && out_dtype != QSA_OUT_F32) return QSA_ERR_INVALID_ARG;
+  if (nq == 0) return QSA_OK;
+  if (!part_o || !part_lse || !out || !lse) return QSA_ERR_INVALID_ARG;
+  if (o_q_stride < 0 || o_split_stride < 0 || lse_q_stride < 0 || lse_split_stride < 0 || (o_q_stride & 3) ||
+      (o_split_stride & 3))
+    return QSA_ERR_INVALID_ARG;
+  const uintptr_t out_align = out_dtype == QSA_OUT_F32 ? 15u : 7u;
+  if ((reinterpret_cast<uintptr_t>(part_o) & 15u) || (reinterpret_cast<uintptr_t>(out) & out_align))
+    return QSA_ERR_INVALID_ARG;
+  const int64_t grid = (int64_t)nq * hq;
+  if (grid > 0x7fffffff) return QSA_ERR_UNSUPPORTED;
+  const CombineArgs a{part_o, part_lse, nsplits, hq, o_q_stride, o_split_stride, lse_q_stride, lse_split_stride, out,
+                      lse};
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return out_dtype == QSA_OUT_F32
+             ? qsa_host::launch(combine_kernel<true>, dim3((unsigned)grid), dim3(kThreads), 0, s, a)
+             : qsa_host::launch(combine_kernel<false>, dim3((unsigned)grid), dim3(kThreads), 0, s, a);
+}
+
 extern "C" int qsa_combine(const float* part_o, const float* part_lse, int32_t nq, int32_t max_splits, int32_t hq,
                            void* out, float* lse, void* stream) {
   if (nq < 0 || max_splits < 1 || hq < 1) return QSA_ERR_INVALID_ARG;
-  if (nq == 0) return QSA_OK;
-  if (!part_o || !part_lse || !out || !lse) return QSA_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(part_o) & 15u) || (reinterpret_cast<uintptr_t>(out) & 7u)) return QSA_ERR_INVALID_ARG;
-  const int64_t grid = (int64_t)nq * hq;
-  if (grid > 0x7fffffff) return QSA_ERR_UNSUPPORTED;
-  return qsa_host::launch(combine_kernel, dim3((unsigned)grid), dim3(kThreads), 0, static_cast<cudaStream_t>(stream),
-                          part_o, part_lse, max_splits, hq, static_cast<__nv_bfloat16*>(out), lse);
+  const int64_t S = max_splits, H = hq;
+  return qsa_combine_strided(part_o, part_lse, nq, max_splits, hq, S * H * kHeadDim, H * kHeadDim, S * H, H, out,
+                             QSA_OUT_BF16, lse, stream);
 }

@@ -65,6 +65,9 @@ def _load() -> ctypes.CDLL:
         "qsa_decode_plan": (ctypes.c_int, [I32, I32, I32, I32, ctypes.POINTER(I32), ctypes.POINTER(I32)]),
         "qsa_sparse_decode": (ctypes.c_int, [PC, P, I32, I32, P, P, P, P, I32, F, I32, I32, P, P, P, P]),
         "qsa_combine": (ctypes.c_int, [P, P, I32, I32, I32, P, P, P]),
+        "qsa_combine_strided": (ctypes.c_int, [P, P, I32, I32, I32, I64, I64, I64, I64, P, I32, P, P]),
+        "qsa_dcp_localize_tokens": (ctypes.c_int, [P, P, I32, I32, I32, I32, P, P, P]),
+        "qsa_dcp_localize_selection": (ctypes.c_int, [P, P, P, I32, I32, I32, I32, I32, P, P, P, P, P]),
         "qsa_sparse_attention_noalloc": (ctypes.c_int, [PC, P, I32, I32, P, P, P, P, I32, F, I32, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
@@ -122,20 +125,27 @@ class PagedCache:
 
     kv_pages is [page][Hkv][16 micro-blocks][2 (K, V)][4 rows][256]: one selected
     micro-block of one KV head is a contiguous run, 4 KiB in BF16 (kv_dtype
-    KV_BF16) or 2 KiB in FP8 e4m3 (KV_FP8_E4M3)."""
+    KV_BF16) or 2 KiB in FP8 e4m3 (KV_FP8_E4M3).  with_kv=False leaves out the
+    main K/V (a selector-only group), with_kc=False the side cache (a K/V-only
+    group, e.g. a DCP rank's shard)."""
 
     def __init__(self, num_pages: int, max_seqs: int, max_pages_per_seq: int, num_kv_heads: int,
-                 block_table: torch.Tensor | None = None, device="cuda", kv_dtype: int = KV_BF16):
+                 block_table: torch.Tensor | None = None, device="cuda", kv_dtype: int = KV_BF16,
+                 with_kv: bool = True, with_kc: bool = True):
         dev = torch.device(device)
         if kv_dtype not in _KV_TORCH:
             raise ValueError(f"kv_dtype must be KV_BF16 or KV_FP8_E4M3, got {kv_dtype}")
         self.num_pages, self.max_seqs, self.max_pages_per_seq, self.num_kv_heads = (
             int(num_pages), int(max_seqs), int(max_pages_per_seq), int(num_kv_heads))
         self.kv_dtype = int(kv_dtype)
+        if not (with_kv or with_kc):
+            raise ValueError("a cache group needs the main K/V, the side cache, or both")
         self.kv_pages = torch.empty((num_pages, num_kv_heads, BLOCKS_PER_PAGE, 2, RATIO, HEAD_DIM),
-                                    dtype=_KV_TORCH[self.kv_dtype], device=dev)
-        self.kc_pages = torch.empty((num_pages, BLOCKS_PER_PAGE, IDX_DIM), dtype=torch.bfloat16, device=dev)
-        self.kc_partial = torch.zeros((max_seqs, IDX_DIM), dtype=torch.float32, device=dev)
+                                    dtype=_KV_TORCH[self.kv_dtype], device=dev) if with_kv else None
+        self.kc_pages = torch.empty((num_pages, BLOCKS_PER_PAGE, IDX_DIM), dtype=torch.bfloat16,
+                                    device=dev) if with_kc else None
+        self.kc_partial = torch.zeros((max_seqs, IDX_DIM), dtype=torch.float32, device=dev) if with_kc else None
+        self.device = dev
         if block_table is None:
             block_table = torch.full((max_seqs, max_pages_per_seq), -1, dtype=torch.int32)
         self.block_table = block_table.to(device=dev, dtype=torch.int32).contiguous()
@@ -144,9 +154,10 @@ class PagedCache:
 
     def struct(self) -> qsa_cache_t:
         if self._struct is None:
-            self._struct = qsa_cache_t(self.kv_pages.data_ptr(), self.kc_pages.data_ptr(),
-                                       self.kc_partial.data_ptr(), self.block_table.data_ptr(), self.num_pages,
-                                       self.max_seqs, self.max_pages_per_seq, self.num_kv_heads, self.kv_dtype)
+            dp = lambda t: None if t is None else t.data_ptr()
+            self._struct = qsa_cache_t(dp(self.kv_pages), dp(self.kc_pages), dp(self.kc_partial),
+                                       self.block_table.data_ptr(), self.num_pages, self.max_seqs,
+                                       self.max_pages_per_seq, self.num_kv_heads, self.kv_dtype)
         return self._struct
 
     def k_view(self) -> torch.Tensor:
@@ -241,6 +252,64 @@ def qsa_combine(part_o, part_lse, out, lse, stream=None):
                                           _stream(stream)))
 
 
+OUT_BF16 = 0
+OUT_F32 = 1
+
+
+def qsa_combine_ranks(part_o, part_lse, out, lse, stream=None):
+    """Merge results laid out split-major: part_o [S][nq][hq][256] fp32 and
+    part_lse [S][nq][hq] (e.g. one fp32 result per DCP rank, gathered rank-major).
+    out: bf16 or fp32 [nq][hq][256]; lse fp32 [nq][hq]."""
+    S, nq, hq = (int(x) for x in part_lse.shape)
+    _req(part_o, "part_o", torch.float32, (S, nq, hq, HEAD_DIM))
+    _req(part_lse, "part_lse", torch.float32, (S, nq, hq))
+    if out.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out must be bf16 or fp32")
+    _req(out, "out", out.dtype, (nq, hq, HEAD_DIM))
+    _req(lse, "lse", torch.float32, (nq, hq))
+    od = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
+    _check("qsa_combine_strided", LIB.qsa_combine_strided(
+        _ptr(part_o), _ptr(part_lse), nq, S, hq, hq * HEAD_DIM, nq * hq * HEAD_DIM, hq, nq * hq, _ptr(out), od,
+        _ptr(lse), _stream(stream)))
+
+
+def qsa_combine_f32(part_o, part_lse, out, lse, stream=None):
+    """qsa_combine with an fp32 result (part_o [nq][S][hq][256]); the result can
+    be one split of a later merge."""
+    nq, S, hq = (int(x) for x in part_lse.shape)
+    _req(part_o, "part_o", torch.float32, (nq, S, hq, HEAD_DIM))
+    _req(part_lse, "part_lse", torch.float32, (nq, S, hq))
+    _req(out, "out", torch.float32, (nq, hq, HEAD_DIM))
+    _req(lse, "lse", torch.float32, (nq, hq))
+    _check("qsa_combine_strided", LIB.qsa_combine_strided(
+        _ptr(part_o), _ptr(part_lse), nq, S, hq, S * hq * HEAD_DIM, hq * HEAD_DIM, S * hq, hq, _ptr(out), OUT_F32,
+        _ptr(lse), _stream(stream)))
+
+
+def qsa_dcp_localize_tokens(seq_id, pos, nranks: int, rank: int, interleave_pages: int, seq_id_local, pos_local,
+                            stream=None):
+    n = int(seq_id.shape[0])
+    for t, nm in ((seq_id, "seq_id"), (pos, "pos"), (seq_id_local, "seq_id_local"), (pos_local, "pos_local")):
+        _req(t, nm, torch.int32, (n,))
+    _check("qsa_dcp_localize_tokens", LIB.qsa_dcp_localize_tokens(
+        _ptr(seq_id), _ptr(pos), n, int(nranks), int(rank), int(interleave_pages), _ptr(seq_id_local),
+        _ptr(pos_local), _stream(stream)))
+
+
+def qsa_dcp_localize_selection(sel, count, q_pos, k: int, nranks: int, rank: int, interleave_pages: int, sel_local,
+                               count_local, q_pos_local, dev_status=None, stream=None):
+    nq = int(q_pos.shape[0])
+    _req(sel, "sel", torch.int32, (nq, k))
+    _req(sel_local, "sel_local", torch.int32, (nq, k))
+    for t, nm in ((count, "count"), (q_pos, "q_pos"), (count_local, "count_local"), (q_pos_local, "q_pos_local")):
+        _req(t, nm, torch.int32, (nq,))
+    if dev_status is not None:
+        _req(dev_status, "dev_status", torch.int32, (1,))
+    _check("qsa_dcp_localize_selection", LIB.qsa_dcp_localize_selection(
+        _ptr(sel), _ptr(count), _ptr(q_pos), nq, int(k), int(nranks), int(rank), int(interleave_pages),
+        _ptr(sel_local), _ptr(count_local), _ptr(q_pos_local), _ptr(dev_status), _stream(stream)))
+
+
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -315,7 +384,7 @@ class Decoder:
 
     def __init__(self, cache: PagedCache, hq: int, max_nq: int, k: int = 512, scale: float = 1.0 / 16.0,
                  target_ctas: int | None = None, chunk_units: int | None = None, scores_ld: int | None = None):
-        dev = cache.kv_pages.device
+        dev = cache.device
         self.cache, self.hq, self.k, self.scale, self.max_nq = cache, hq, k, scale, max_nq
         if target_ctas is None:
             target_ctas = torch.cuda.get_device_properties(dev).multi_processor_count

@@ -25,7 +25,7 @@ def test_library_exports_every_declared_symbol():
     lib = ctypes.CDLL(qsa.LIB_PATH)
     for n in header_functions():
         assert hasattr(lib, n), n
-    assert qsa.ABI_VERSION == 3
+    assert qsa.ABI_VERSION == 4
     assert qsa.status_string(0) == "QSA_OK" and qsa.status_string(-3) == "QSA_ERR_CUDA"
 
 
@@ -65,6 +65,26 @@ def test_host_validation_returns_before_any_cuda_call():
     assert L.qsa_index_scores(cp, None, fake, fake, fake, 1, fake, 16, None, None) == -1
     assert L.qsa_combine(ctypes.c_void_p(0x1004), fake, 1, 4, 16, fake, fake, None) == -1  # misaligned
     assert L.qsa_combine(fake, fake, 1, 0, 16, fake, fake, None) == -1
+    # strided merge: output type, 16-byte strides of part_o, fp32 output alignment
+    assert L.qsa_combine_strided(fake, fake, 1, 2, 4, 2048, 1024, 8, 4, fake, 2, fake, None) == -1
+    assert L.qsa_combine_strided(fake, fake, 1, 2, 4, 2046, 1024, 8, 4, fake, 0, fake, None) == -1
+    assert L.qsa_combine_strided(fake, fake, 1, 2, 4, 2048, 1024, 8, 4, ctypes.c_void_p(0x1008), 1, fake, None) == -1
+    assert L.qsa_combine_strided(fake, fake, 0, 2, 4, 2048, 1024, 8, 4, fake, 1, fake, None) == 0
+    # DCP localisation: the shard must be well formed
+    assert L.qsa_dcp_localize_tokens(fake, fake, 4, 2, 2, 1, fake, fake, None) == -1
+    assert L.qsa_dcp_localize_tokens(fake, fake, 4, 0, 0, 1, fake, fake, None) == -1
+    assert L.qsa_dcp_localize_tokens(fake, fake, 4, 2, 1, 0, fake, fake, None) == -1
+    assert L.qsa_dcp_localize_tokens(fake, fake, 0, 2, 1, 1, fake, fake, None) == 0
+    assert L.qsa_dcp_localize_selection(fake, fake, fake, 1, 16, 2, -1, 1, fake, fake, fake, None, None) == -1
+    assert L.qsa_dcp_localize_selection(fake, fake, fake, 1, 4096, 2, 0, 1, fake, fake, fake, None, None) == -1
+    # a cache group needs at least one of main K/V and side cache
+    empty = qsa.qsa.qsa_cache_t(None, None, 0x1000, 0x1000, 10, 2, 4, 2)
+    assert L.qsa_append_kv(ctypes.byref(empty), fake, fake, fake, fake, fake, 5, None, None) == -1
+    kv_only = qsa.qsa.qsa_cache_t(0x1000, None, None, 0x1000, 10, 2, 4, 2)
+    assert L.qsa_index_scores(ctypes.byref(kv_only), fake, fake, fake, fake, 1, fake, 16, None, None) == -1
+    kc_only = qsa.qsa.qsa_cache_t(None, 0x1000, 0x1000, 0x1000, 10, 2, 4, 2)
+    assert L.qsa_sparse_decode(ctypes.byref(kc_only), fake, 1, 16, fake, fake, fake, fake, 16, 0.0625, 16, 4, fake,
+                               fake, None, None) == -1
     # K/V storage types: BF16 and FP8 e4m3 only
     bad = qsa.qsa.qsa_cache_t(0x1000, 0x1000, 0x1000, 0x1000, 10, 2, 4, 2, 7)
     bp = ctypes.byref(bad)
