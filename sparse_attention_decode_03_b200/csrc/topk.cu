@@ -40,7 +40,6 @@ struct TopkArgs {
   int64_t ld;
   const int32_t* q_pos;
   int32_t K;
-  int32_t fast_cap;  // blocks per query the shared-memory path holds
   int32_t* sel;
   int32_t* count;
   int32_t* st;
@@ -468,7 +467,7 @@ extern "C" int qsa_topk_blocks(const float* scores, int64_t scores_ld, const int
   if (nq < 0 || k < 0 || k > QSA_MAX_TOPK || scores_ld < 1) return QSA_ERR_INVALID_ARG;
   if (nq == 0) return QSA_OK;
   if (!scores || !q_pos || !count || (k > 0 && !sel)) return QSA_ERR_INVALID_ARG;
-  TopkArgs a{scores, scores_ld, q_pos, k, 0, sel, count, dev_status};
+  TopkArgs a{scores, scores_ld, q_pos, k, sel, count, dev_status};
   const int smem = (int)sizeof(TopkSmem);
   if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
     (void)cudaGetLastError();

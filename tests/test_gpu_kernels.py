@@ -498,3 +498,34 @@ def test_step_io_staging_and_readback():
     assert nbytes == wl.nq * wl.hq * 256 * 2 + wl.nq * wl.hq * 4
     assert torch.equal(host[1][:wl.nq].view(torch.int16), dec2.out[:wl.nq].cpu().view(torch.int16))
     assert torch.all(host[1][wl.nq:] == 0)
+
+
+@pytest.mark.parametrize("hq,hkv,k,L", [
+    (16, 1, 2048, 4 * 2300 + 2),    # the largest group (16 Q heads per KV head) and the largest budget
+    (2, 2, 2048, 4 * 2048 + 3),     # one Q head per KV head; budget = every complete block but none spare
+    (32, 2, 700, 4 * 3000),         # group 16 at two KV heads, no tail
+])
+def test_decode_limits_budget_and_group(hq, hkv, k, L):
+    wl = dataclasses.replace(C.shrink(C.get("quarter"), [L - 1], k_top=k, page_perm=True), hq=hq, hkv=hkv)
+    cache, dec, st = run_step(wl, k=k)
+    assert st == 0
+    assert int(dec.count[0]) == min(k, L // 4)
+    _check_decode(wl, dec, [0], k=k)
+
+
+def test_noalloc_call_on_an_fp8_cache():
+    wl = dataclasses.replace(C.shrink(C.get("long"), [4000, 2500], k_top=256, page_perm=True), kv_fp8=True)
+    cache, dec, st = run_step(wl, k=256)
+    assert st == 0
+    s2 = _status()
+    out = torch.empty_like(dec.out[:wl.nq])
+    lse = torch.empty_like(dec.lse[:wl.nq])
+    inp = H.step_inputs(wl)
+    qsa.qsa_sparse_attention_noalloc(cache, inp["q"], inp["q_seq"], inp["q_pos"], dec.sel[:wl.nq], dec.count[:wl.nq],
+                                     256, wl.scale, dec.chunk_units, out, lse, s2)
+    torch.cuda.synchronize()
+    assert int(s2.item()) == 0
+    assert torch.equal(out.view(torch.int16), dec.out[:wl.nq].view(torch.int16))
+    for row in range(wl.nq):
+        ref = R.expect_query(wl, row, k=256)
+        R.assert_close(out[row].float().cpu().numpy(), ref["o"], f"noalloc fp8 row {row}")
