@@ -21,8 +21,12 @@ namespace {
 using namespace qsa;
 
 constexpr int kWarps = 8;
-constexpr int kPagesPerWarp = 4;
-constexpr int kPagesPerCta = kWarps * kPagesPerWarp;  // 32 pages = 512 blocks = 128 KiB
+// Each warp scores a run of pages_per_warp pages (2 at a time), a CTA 8 such
+// runs.  The host sizes the run (4 to 16 pages) so the grid keeps about six
+// waves of resident CTAs: fewer, longer CTAs when the block table is wide
+// and many of its chunks hold no pages of a shorter query, more and shorter
+// ones when every chunk is full.
+constexpr int kMinPagesPerWarp = 4, kMaxPagesPerWarp = 16;
 
 struct ScoreArgs {
   const __nv_bfloat16* kc;
@@ -35,6 +39,7 @@ struct ScoreArgs {
   float* scores;
   int64_t ld;
   int32_t chunks_per_query;
+  int32_t pages_per_warp;
   int32_t* st;
 };
 
@@ -60,7 +65,8 @@ __global__ void __launch_bounds__(kWarps * 32) index_scores_kernel(ScoreArgs a) 
     nb = a.ld;
   }
   const int npg = (int)((nb + kBlocksPerPage - 1) / kBlocksPerPage);
-  const int pg0 = chunk * kPagesPerCta + warp * kPagesPerWarp;
+  const int ppw = a.pages_per_warp;
+  const int pg0 = chunk * (kWarps * ppw) + warp * ppw;
   if (pg0 >= npg) return;
 
   // B fragments: indexer query head g, chunks 4i+t of its 128 dims.
@@ -72,11 +78,11 @@ __global__ void __launch_bounds__(kWarps * 32) index_scores_kernel(ScoreArgs a) 
   const float w1 = a.w[q * kIdxHeads + 2 * t + 1];
 
   int myphys = -1;
-  if (lane < kPagesPerWarp && pg0 + lane < npg) myphys = a.bt[(int64_t)seq * a.mpps + pg0 + lane];
+  if (lane < ppw && pg0 + lane < npg) myphys = a.bt[(int64_t)seq * a.mpps + pg0 + lane];
   float* srow = a.scores + (size_t)q * a.ld;
 
 #pragma unroll
-  for (int pp = 0; pp < kPagesPerWarp; pp += 2) {
+  for (int pp = 0; pp < ppw; pp += 2) {
     uint4 ra[2][4], rb[2][4];
     int phys[2];
     bool ok[2];
@@ -553,7 +559,24 @@ extern "C" int qsa_index_scores(const qsa_cache_t* cache, const void* q_idx, con
   int64_t max_pages = cache->max_pages_per_seq;
   const int64_t ld_pages = (scores_ld + kBlocksPerPage - 1) / kBlocksPerPage;
   if (ld_pages < max_pages) max_pages = ld_pages;
-  a.chunks_per_query = (int32_t)((max_pages + kPagesPerCta - 1) / kPagesPerCta);
+  // run length: the longest that still leaves about six waves of resident CTAs
+  int ppw = kMinPagesPerWarp;
+  {
+    int dev = 0, sms = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, index_scores_kernel, kWarps * 32, 0) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return QSA_ERR_CUDA;
+    }
+    const int64_t slots = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
+    while (ppw < kMaxPagesPerWarp) {
+      const int64_t ctas = (int64_t)nq * ((max_pages + kWarps * 2 * ppw - 1) / (kWarps * 2 * ppw));
+      if (ctas < 6 * slots) break;
+      ppw *= 2;
+    }
+  }
+  a.pages_per_warp = ppw;
+  a.chunks_per_query = (int32_t)((max_pages + kWarps * ppw - 1) / (kWarps * ppw));
   a.st = dev_status;
   const int64_t grid = (int64_t)nq * a.chunks_per_query;
   if (grid > 0x7fffffff) return QSA_ERR_UNSUPPORTED;
