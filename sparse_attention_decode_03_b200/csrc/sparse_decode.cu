@@ -76,7 +76,8 @@ struct Lay {
   static constexpr int kOffQ = kOffRing + kStages * kStageBytes;
   static constexpr int kOffComb = kOffQ + kQBufBytes;
   static constexpr int kOffML = kOffComb + kCombBytes;
-  static constexpr int kOffDescOff = kOffML + kPairs * 16 * 2 * 4;
+  static constexpr int kOffX = kOffML + kPairs * 16 * 2 * 4;              // S exchange: [pair][parity][half][lane][8]
+  static constexpr int kOffDescOff = kOffX + kPairs * 2 * 2 * 32 * 8 * 4;
   static constexpr int kOffDescRows = kOffDescOff + kDescSlots * kBatch * 8;
   static constexpr int kOffMeta = kOffDescRows + kDescSlots * kBatch * 4;
   static constexpr int kOffBar = (kOffMeta + kStages * 4 + 7) & ~7;
@@ -98,13 +99,14 @@ struct Lay {
   constexpr int kOffQ = LY::kOffQ;                          \
   constexpr int kOffComb = LY::kOffComb;                    \
   constexpr int kOffML = LY::kOffML;                        \
+  constexpr int kOffX = LY::kOffX;                          \
   constexpr int kOffDescOff = LY::kOffDescOff;              \
   constexpr int kOffDescRows = LY::kOffDescRows;            \
   constexpr int kOffMeta = LY::kOffMeta;                    \
   constexpr int kOffBar = LY::kOffBar;                      \
   constexpr int kOffAbort = LY::kOffAbort;                  \
   (void)kStages; (void)kHalfBytes; (void)kUnitBytes; (void)kSlotStride; (void)kStageBytes; (void)kOffRing; \
-  (void)kOffQ; (void)kOffComb; (void)kOffML; (void)kOffDescOff; (void)kOffDescRows; (void)kOffMeta;      \
+  (void)kOffQ; (void)kOffComb; (void)kOffML; (void)kOffX; (void)kOffDescOff; (void)kOffDescRows; (void)kOffMeta;      \
   (void)kOffBar; (void)kOffAbort
 // full barrier: the 32 lanes' copy-completion arrivals + the owning copy warp's
 // lane 0, whose plain (release) arrival publishes the stage's row mask
@@ -497,19 +499,22 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
       const uint32_t mask = meta[stage];
       const uint32_t kb = ring + stage * kStageBytes;
 
-      // ---- S = Q K^T : two n-tiles of 8 tokens, k = 256 dims in 16 steps (both warps of the pair)
+      // ---- S = Q K^T : two n-tiles of 8 tokens; this warp sums its half of the
+      // 256 dims (k-steps 8 half .. 8 half + 7) and the pair exchanges the partial
+      // sums in shared memory (a + b == b + a, so both warps hold the same S)
       float sa[2][4], sb[2][4];
 #pragma unroll
       for (int j = 0; j < 2; ++j)
 #pragma unroll
         for (int c = 0; c < 4; ++c) sa[j][c] = sb[j][c] = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int ii = 0; ii < 4; ++ii) {
+        const int i = 4 * half + ii;
         const uint4 qa = lds128(qb + gq * kQRowStride + (4 * i + tq) * 16);
         const uint4 qc = lds128(qb + (gq + 8) * kQRowStride + (4 * i + tq) * 16);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          float(&acc)[4] = (i & 1) ? sb[j] : sa[j];
+          float(&acc)[4] = (ii & 1) ? sb[j] : sa[j];
           if constexpr (F8) {
             const uint4 kk = e4m3x8_to_f16x8(lds64(kb + k_off + j * 2 * kRowBytes + i * 32));
             mma_f16_16816(acc, qa.x, qc.x, qa.y, qc.y, kk.x, kk.y);
@@ -520,6 +525,23 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
             mma_bf16_16816(acc, qa.z, qc.z, qa.w, qc.w, kk.z, kk.w);
           }
         }
+      }
+      {
+        float* xb = reinterpret_cast<float*>(smem + kOffX) + ((cp * 2 + (int)((T / kPairs) & 1)) * 2) * 256;
+        float4* mine = reinterpret_cast<float4*>(xb + (half * 32 + lane) * 8);
+        const float4 p0 = make_float4(sa[0][0] + sb[0][0], sa[0][1] + sb[0][1], sa[0][2] + sb[0][2], sa[0][3] + sb[0][3]);
+        const float4 p1 = make_float4(sa[1][0] + sb[1][0], sa[1][1] + sb[1][1], sa[1][2] + sb[1][2], sa[1][3] + sb[1][3]);
+        mine[0] = p0;
+        mine[1] = p1;
+        named_bar_sync(2 + cp, 64);  // the pair's two warps
+        const float4* other = reinterpret_cast<const float4*>(xb + ((1 - half) * 32 + lane) * 8);
+        const float4 o0 = other[0], o1 = other[1];
+        sa[0][0] = p0.x + o0.x; sa[0][1] = p0.y + o0.y; sa[0][2] = p0.z + o0.z; sa[0][3] = p0.w + o0.w;
+        sa[1][0] = p1.x + o1.x; sa[1][1] = p1.y + o1.y; sa[1][2] = p1.z + o1.z; sa[1][3] = p1.w + o1.w;
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) sb[j][c] = 0.f;
       }
       // ---- mask, online softmax (base-2 logits)
       float z[2][4];
