@@ -17,9 +17,10 @@
 // chunk is a "segment"; each segment yields one split partial.
 //
 // CTA = 8 consumer warps + 2 copy warps + a lookup warp, 1 CTA per SM.
-//   lookup warp: walks the CTA's units 32 at a time (selection -> page table)
-//     and writes their source offsets into a 3-batch descriptor queue, so the
-//     dependent selection and page-table loads run ahead of the copies.
+//   lookup warp: walks the CTA's units 32 at a time (selection -> page table),
+//     four batches per round, and writes their source offsets into an 8-batch
+//     descriptor queue, so the dependent selection and page-table loads run
+//     ahead of the copies.
 //   copy warps: tile T (4 units) belongs to copy warp T % 2, which moves each
 //     unit's 4 KiB with 16-byte cp.async copies (every lane 8 per unit) into
 //     an 8-stage shared-memory ring; each lane then arrives on the stage's
@@ -28,12 +29,16 @@
 //     gathers stayed near half the HBM rate on B200; spreading the issue over
 //     the lanes of more warps is what raises the gather rate.
 //   consumers: 4 pairs of warps; tile T (16 tokens) belongs to pair T % 4.
-//     Both warps of a pair compute S = Q K^T for the tile and the online
-//     softmax (mma.sync m16n8k16, M = 16 Q-head rows of the KV group, fp32
-//     accumulate); each accumulates O += P V for its half of the 256 output
-//     dims, which halves the accumulator registers and lets 8 consumer warps
-//     keep the copies fed.  At the end of a segment the 4 pairs merge their
-//     (m, l, O) in two rounds through shared memory and write the partial.
+//     Each warp of a pair computes S = Q K^T over its half of the 256 dims
+//     (mma.sync m16n8k16, M = 16 Q-head rows of the KV group, fp32
+//     accumulate) and the pair swaps the partial sums through shared memory,
+//     so both hold the whole S; both run the same online softmax, and each
+//     accumulates O += P V for its half of the 256 output dims, which halves
+//     the accumulator registers and lets 8 consumer warps keep the copies
+//     fed.  At the end of a segment the 4 pairs merge their (m, l, O) in two
+//     steps through shared memory and write the partial.
+// FP8 e4m3 K/V (template F8): 2 KiB units, a 16-stage ring of 8 KiB tiles, K
+// and V widened to FP16 in registers, FP16 MMAs.
 // Shared-memory layouts are skewed so that every 16-byte fragment read is
 // bank-conflict free (micro-block slots 4128 B apart, Q rows 576 B apart).
 #include "qsa_common.cuh"
@@ -728,7 +733,7 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
         }
       }
     };
-    // round 1: pairs 2, 3 hand their O to pairs 0, 1; round 2: pair 1 to pair 0
+    // merge step 1: pairs 2, 3 hand their O to pairs 0, 1; step 2: pair 1 to pair 0
     if (cp >= 2) store_rows(comb + (cp - 2) * 16 * kCombRow, kCombRow);
     named_bar_sync(kBarConsumers, kConsumerThreads);
     if (cp < 2) add_rows(comb + cp * 16 * kCombRow);
