@@ -32,8 +32,10 @@ namespace {
 
 using namespace qsa;
 
-constexpr int kThreads = 1024;
-constexpr int kWarps = kThreads / 32;
+// Block sizes: 1024 threads (few queries: one query's latency is the step's)
+// or 256 threads (many queries: more CTAs resident per SM, more throughput).
+// Every function below is templated on the block size kThreads.
+constexpr int kThreadsLarge = 1024, kThreadsSmall = 256;
 
 struct TopkArgs {
   const float* scores;
@@ -47,8 +49,10 @@ struct TopkArgs {
 
 // Block-wide: find the bin b (scanning from the top) with
 // sum_{i > b} hist[i] < remaining <= sum_{i >= b} hist[i].
+template <int kThreads>
 __device__ void find_bin(const uint32_t* hist, int nbins, uint32_t remaining, uint32_t* wsum, int* out_bin,
                          uint32_t* out_above) {
+  constexpr int kWarps = kThreads / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int per = nbins >= kThreads ? nbins / kThreads : 1;
   const int lo = tid * per;
@@ -82,6 +86,7 @@ __device__ void find_bin(const uint32_t* hist, int nbins, uint32_t remaining, ui
 
 constexpr int kUnroll = 8;
 
+template <int kThreads>
 __device__ __forceinline__ void load_keys(const float* s, int i0, int n, uint32_t (&key)[kUnroll]) {
 #pragma unroll
   for (int u = 0; u < kUnroll; ++u) {
@@ -91,8 +96,10 @@ __device__ __forceinline__ void load_keys(const float* s, int i0, int n, uint32_
 }
 
 // General path: exact K-th key by three radix passes, then ordered compaction.
+template <int kThreads>
 __device__ void topk_general(const float* s, int n, int K, int32_t* out, uint32_t* hist, uint32_t* wsum,
                              uint32_t* wgt, uint32_t* weq, int* s_bin, uint32_t* s_above) {
+  constexpr int kWarps = kThreads / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t prefix = 0, mask = 0, remaining = (uint32_t)K;
   const int shifts[3] = {20, 8, 0};
@@ -104,13 +111,13 @@ __device__ void topk_general(const float* s, int n, int K, int32_t* out, uint32_
     __syncthreads();
     for (int i0 = tid; i0 < n; i0 += kThreads * kUnroll) {
       uint32_t key[kUnroll];
-      load_keys(s, i0, n, key);
+      load_keys<kThreads>(s, i0, n, key);
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u)
         if (i0 + u * kThreads < n && (key[u] & mask) == prefix) atomicAdd(&hist[(key[u] >> sh) & (nbins - 1)], 1u);
     }
     __syncthreads();
-    find_bin(hist, nbins, remaining, wsum, s_bin, s_above);
+    find_bin<kThreads>(hist, nbins, remaining, wsum, s_bin, s_above);
     prefix |= (uint32_t)*s_bin << sh;
     mask |= (uint32_t)(nbins - 1) << sh;
     remaining -= *s_above;
@@ -162,6 +169,7 @@ constexpr int kCap = 256;       // candidates one warp's list holds
 constexpr int kWin = 12;        // radix window bits
 constexpr int kWinBins = 1 << kWin;
 
+template <int kWarps>
 struct TopkSmem {
   uint32_t ckey[kWarps][kCap];  // candidate keys, per warp, in index order
   uint32_t cidx[kWarps][kCap];  // their block indices
@@ -182,7 +190,9 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool live
 }
 
 // Block-wide min and max of one value per thread.
+template <int kThreads>
 __device__ __forceinline__ void block_minmax(uint32_t& mn, uint32_t& mx, uint32_t* red) {
+  constexpr int kWarps = kThreads / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   mn = __reduce_min_sync(0xffffffffu, mn);
   mx = __reduce_max_sync(0xffffffffu, mx);
@@ -191,14 +201,17 @@ __device__ __forceinline__ void block_minmax(uint32_t& mn, uint32_t& mx, uint32_
     red[kWarps + warp] = mx;
   }
   __syncthreads();
-  mn = __reduce_min_sync(0xffffffffu, red[lane]);
-  mx = __reduce_max_sync(0xffffffffu, red[kWarps + lane]);
+  mn = __reduce_min_sync(0xffffffffu, lane < kWarps ? red[lane] : 0xffffffffu);
+  mx = __reduce_max_sync(0xffffffffu, lane < kWarps ? red[kWarps + lane] : 0u);
   __syncthreads();
 }
 
 // The bin b of hist[0..nbins) (counting from the top) with
 // sum_{>b} < remaining <= sum_{>=b}; *above = sum_{>b}.  Same result in every thread.
-__device__ int top_bin(const uint32_t* hist, int nbins, uint32_t remaining, TopkSmem& S, uint32_t* above) {
+template <int kThreads>
+__device__ int top_bin(const uint32_t* hist, int nbins, uint32_t remaining, TopkSmem<kThreads / 32>& S,
+                       uint32_t* above) {
+  constexpr int kWarps = kThreads / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int per = (nbins + kThreads - 1) / kThreads;
   const int b0 = tid * per;
@@ -214,7 +227,7 @@ __device__ int top_bin(const uint32_t* hist, int nbins, uint32_t remaining, Topk
   if (lane == 0) S.wsum[warp] = suf;
   __syncthreads();
   // sum of the totals of the warps above mine: a suffix scan across lanes
-  const uint32_t wt = S.wsum[lane];
+  const uint32_t wt = lane < kWarps ? S.wsum[lane] : 0u;
   uint32_t wsuf = wt;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
@@ -258,7 +271,8 @@ __device__ __forceinline__ void load_batch(const float* s, int c0, int hi, bool 
 }
 
 // Append lane's flagged keys (f0..f3 of idx0..idx0+3) to this warp's list, in index order.
-__device__ __forceinline__ void append4(TopkSmem& S, int warp, uint32_t& cnt, const uint32_t (&k)[4], int idx0,
+template <int kWarps>
+__device__ __forceinline__ void append4(TopkSmem<kWarps>& S, int warp, uint32_t& cnt, const uint32_t (&k)[4], int idx0,
                                         const bool (&f)[4]) {
   const int lane = threadIdx.x & 31;
   const uint32_t nc = (uint32_t)f[0] + f[1] + f[2] + f[3];
@@ -282,11 +296,14 @@ __device__ __forceinline__ void append4(TopkSmem& S, int warp, uint32_t& cnt, co
   cnt += tot;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) topk_kernel(TopkArgs a) {
+template <int kThreads>
+__global__ void __launch_bounds__(kThreads, kThreads == kThreadsLarge ? 1 : 4) topk_kernel(TopkArgs a) {
+  constexpr int kWarps = kThreads / 32;
+  constexpr int kSPer = kSample / kThreads;  // sample keys per thread
   pdl_launch_dependents();
   pdl_wait_previous();
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  TopkSmem& S = *reinterpret_cast<TopkSmem*>(smem_raw);
+  TopkSmem<kWarps>& S = *reinterpret_cast<TopkSmem<kWarps>*>(smem_raw);
   const int q = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int p = a.q_pos[q];
@@ -314,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(TopkArgs a) {
   // Each warp owns a contiguous segment of the row (a multiple of 128 keys).
   // Its first kBatch x 128 keys are loaded now, so that their latency hides
   // behind the threshold phase.
-  const int seg = (int)(((int64_t)n + 32 * 128 - 1) / (32 * 128)) * 128;
+  const int seg = (int)(((int64_t)n + kWarps * 128 - 1) / (kWarps * 128)) * 128;
   const int w_lo = min(n, warp * seg), w_hi = min(n, w_lo + seg);
   const bool vec = (reinterpret_cast<uintptr_t>(s) & 15u) == 0;
   float4 v[kBatch];
@@ -322,10 +339,18 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(TopkArgs a) {
 
   // ---- 1. threshold T0 from a regular sample
   const int ns = min(n, kSample);
-  const bool live_s = tid < ns;
-  const uint32_t ks = live_s ? float_key(__ldg(s + (int64_t)tid * n / ns)) : 0u;
-  uint32_t smin = live_s ? ks : 0xffffffffu, smax = live_s ? ks : 0u;
-  block_minmax(smin, smax, S.red);
+  uint32_t ks[kSPer];
+  uint32_t smin = 0xffffffffu, smax = 0u;
+#pragma unroll
+  for (int u = 0; u < kSPer; ++u) {
+    const int i = u * kThreads + tid;
+    ks[u] = i < ns ? float_key(__ldg(s + (int64_t)i * n / ns)) : 0u;
+    if (i < ns) {
+      smin = min(smin, ks[u]);
+      smax = max(smax, ks[u]);
+    }
+  }
+  block_minmax<kThreads>(smin, smax, S.red);
   uint32_t r;
   if (ns == n) {
     r = (uint32_t)K;
@@ -341,10 +366,11 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(TopkArgs a) {
     const uint32_t mhi = hb >= 31 ? 0u : ~((2u << hb) - 1u);
     for (int i = tid; i < nbins; i += kThreads) S.hist[i] = 0;
     __syncthreads();
-    hist_add(S.hist, (ks >> wlo) & (uint32_t)(nbins - 1), live_s);
+#pragma unroll
+    for (int u = 0; u < kSPer; ++u) hist_add(S.hist, (ks[u] >> wlo) & (uint32_t)(nbins - 1), u * kThreads + tid < ns);
     __syncthreads();
     uint32_t above;
-    const int b = top_bin(S.hist, nbins, r, S, &above);
+    const int b = top_bin<kThreads>(S.hist, nbins, r, S, &above);
     T0 = (smin & mhi) | ((uint32_t)b << wlo);
   }
 
@@ -370,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(TopkArgs a) {
     overflow |= S.wcnt[w] > kCap;
   }
   if (overflow || total < (uint32_t)K) {  // block-uniform
-    topk_general(s, n, K, out, S.hist, S.wsum, S.wgt, S.weq, &S.bin, &S.above);
+    topk_general<kThreads>(s, n, K, out, S.hist, S.wsum, S.wgt, S.weq, &S.bin, &S.above);
     return;
   }
   const uint32_t mycnt = S.wcnt[warp];
@@ -384,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(TopkArgs a) {
     cmin = min(cmin, ck[j]);
     cmax = max(cmax, ck[j]);
   }
-  block_minmax(cmin, cmax, S.red);
+  block_minmax<kThreads>(cmin, cmax, S.red);
   uint32_t T = cmin, M = 0xffffffffu, remaining = (uint32_t)K;
   int hb = cmin == cmax ? -1 : 31 - __clz(cmin ^ cmax);
   if (hb >= 0) {
@@ -402,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(TopkArgs a) {
     }
     __syncthreads();
     uint32_t above;
-    const int b = top_bin(S.hist, nbins, remaining, S, &above);
+    const int b = top_bin<kThreads>(S.hist, nbins, remaining, S, &above);
     const uint32_t in_bin = S.hist[b];
     remaining -= above;
     T |= (uint32_t)b << wlo;
@@ -427,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(TopkArgs a) {
   }
   __syncthreads();
   if (warp == 0) {  // warp totals -> ties before each warp, first output slot of each warp
-    const uint32_t ew = S.weq[lane], gw = S.wgt[lane];
+    const uint32_t ew = lane < kWarps ? S.weq[lane] : 0u, gw = lane < kWarps ? S.wgt[lane] : 0u;
     uint32_t einc = ew;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -442,8 +468,10 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(TopkArgs a) {
       const uint32_t x = __shfl_up_sync(0xffffffffu, tinc, d);
       if (lane >= d) tinc += x;
     }
-    S.weqb[lane] = eqb;
-    S.wslot[lane] = tinc - take;
+    if (lane < kWarps) {
+      S.weqb[lane] = eqb;
+      S.wslot[lane] = tinc - take;
+    }
   }
   __syncthreads();
   uint32_t eqb = S.weqb[warp], slot = S.wslot[warp];
@@ -460,6 +488,17 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(TopkArgs a) {
   }
 }
 
+template <int kThreads>
+int launch_topk(const TopkArgs& a, int32_t nq, void* stream) {
+  const int smem = (int)sizeof(TopkSmem<kThreads / 32>);
+  if (cudaFuncSetAttribute(topk_kernel<kThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QSA_ERR_CUDA;
+  }
+  return qsa_host::launch(topk_kernel<kThreads>, dim3((unsigned)nq), dim3(kThreads), (size_t)smem,
+                          static_cast<cudaStream_t>(stream), a);
+}
+
 }  // namespace
 
 extern "C" int qsa_topk_blocks(const float* scores, int64_t scores_ld, const int32_t* q_pos, int32_t nq, int32_t k,
@@ -468,11 +507,13 @@ extern "C" int qsa_topk_blocks(const float* scores, int64_t scores_ld, const int
   if (nq == 0) return QSA_OK;
   if (!scores || !q_pos || !count || (k > 0 && !sel)) return QSA_ERR_INVALID_ARG;
   TopkArgs a{scores, scores_ld, q_pos, k, sel, count, dev_status};
-  const int smem = (int)sizeof(TopkSmem);
-  if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
     (void)cudaGetLastError();
     return QSA_ERR_CUDA;
   }
-  return qsa_host::launch(topk_kernel, dim3((unsigned)nq), dim3(kThreads), (size_t)smem,
-                          static_cast<cudaStream_t>(stream), a);
+  // few queries (at most two 1024-thread CTAs per SM): the large block, lowest latency per query;
+  // many: 256-thread blocks, several resident per SM, more queries in flight
+  const bool large = (int64_t)nq <= 2 * (int64_t)sms;
+  return large ? launch_topk<kThreadsLarge>(a, nq, stream) : launch_topk<kThreadsSmall>(a, nq, stream);
 }

@@ -228,15 +228,20 @@ def _topk_rows(kind, n, gen):
     raise ValueError(kind)
 
 
+@pytest.mark.parametrize("nrows", [2, 300])
 @pytest.mark.parametrize("kind", ["random", "ascending", "descending", "ties", "neg_inf", "hot_tail"])
 @pytest.mark.parametrize("n,k,pad", [(513, 512, 0), (1024, 512, 3), (1025, 1, 0), (4095, 2048, 1),
                                      (32768, 512, 0), (65536, 512, 5), (100000, 512, 0)])
-def test_topk_rows_match_oracle_on_every_path(kind, n, k, pad):
+def test_topk_rows_match_oracle_on_every_path(kind, n, k, pad, nrows):
     """Sampled-threshold path (random rows) and its fallback (sorted rows, heavy
     ties, crowded tails overflow a warp's candidate list), aligned and
-    misaligned row strides, -inf scores, rows of 513 .. 100,000 blocks."""
+    misaligned row strides, -inf scores, rows of 513 .. 100,000 blocks; with
+    few queries (1024-thread blocks) and many (300 rows: 256-thread blocks)."""
+    if nrows > 2 and n > 32768:
+        pytest.skip("the many-query form is covered up to 32,768 blocks per row")
     gen = torch.Generator().manual_seed(n * 7 + k + pad)
     rows = [_topk_rows(kind, n, gen), _topk_rows("random", n, gen)]
+    rows += [rows[i % 2] if i % 5 else _topk_rows(kind, n, gen) for i in range(2, nrows)]
     ld = n + pad
     scores = torch.full((len(rows), ld), float("nan"), dtype=torch.float32)
     for i, r in enumerate(rows):
@@ -248,10 +253,15 @@ def test_topk_rows_match_oracle_on_every_path(kind, n, k, pad):
     qsa.qsa_topk_blocks(scores.cuda(), q_pos, k, sel, cnt, st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
+    sel_h, cnt_h = sel.cpu().numpy(), cnt.cpu().numpy()
+    refs = {}
     for i, r in enumerate(rows):
-        ref = O.select_blocks(r.double().numpy(), k)
-        assert int(cnt[i]) == len(ref)
-        assert np.array_equal(sel[i].cpu().numpy()[:len(ref)], ref), f"{kind} row {i}"
+        key = id(r)
+        if key not in refs:
+            refs[key] = O.select_blocks(r.double().numpy(), k)
+        ref = refs[key]
+        assert int(cnt_h[i]) == len(ref)
+        assert np.array_equal(sel_h[i][:len(ref)], ref), f"{kind} row {i}"
 
 
 # ---------------------------------------------------------------- attention
