@@ -15,9 +15,11 @@
  *   a lightweight indexer compresses keys into micro-blocks of 4 tokens and
  *   scores every block against the query; the best 512 blocks (about 2,048
  *   token positions) are kept; softmax and value aggregation then run over the
- *   uncompressed BF16 K and V (head dim 256, GQA) at those positions only; the
- *   attention is split over KV chunks and merged with log-sum-exp (the
- *   single-GPU analogue of the cross-rank combine of [DCP]).
+ *   uncompressed K and V (BF16, or FP8 e4m3; head dim 256, GQA) at those
+ *   positions only; the attention is split over KV chunks and merged with
+ *   log-sum-exp (on one GPU the analogue of the cross-rank combine of [DCP];
+ *   across GPUs the qsa_dcp_* calls shard the K/V by context and the same
+ *   merge combines the ranks).
  * Fixed readings where the pages are silent: kc_j = sum of the 4 tokens'
  * indexer keys (fp32, token order, stored BF16 round-to-nearest-even);
  * s_j = sum_h w_h * ReLU(q_idx,h . kc_j) with 8 indexer heads of dim 128; ties
@@ -37,7 +39,8 @@
  *    sequence id, position, selection index or count.  The offending read is
  *    skipped (masked); kernels never trap.  The caller clears and reads it.
  *  - All outputs are deterministic: no floating-point atomics.
- *  - Tensors are dense row-major with the shapes given; no strides.
+ *  - Tensors are dense row-major with the shapes given; no strides (except
+ *    qsa_combine_strided, which takes them explicitly).
  */
 #ifndef QSA_H
 #define QSA_H
