@@ -132,7 +132,7 @@ QSA_API const char* qsa_status_string(int status);
 
 /* ABI version of this header (bumped on any signature change). */
 QSA_API int qsa_abi_version(void);
-#define QSA_ABI_VERSION 4
+#define QSA_ABI_VERSION 5
 
 /*
  * qsa_append_kv -- write n new tokens into the cache group.
@@ -180,6 +180,41 @@ QSA_API int qsa_index_scores(const qsa_cache_t* cache, const void* q_idx, const 
  */
 QSA_API int qsa_topk_blocks(const float* scores, int64_t scores_ld, const int32_t* q_pos, int32_t nq, int32_t k,
                     int32_t* sel, int32_t* count, int32_t* dev_status, void* stream);
+
+/*
+ * qsa_index_topk -- qsa_index_scores followed by qsa_topk_blocks, in one
+ * kernel: the same scores (bit for bit) and the same selections and counts.
+ * The score row of a query stays in on-chip shared memory, spread over a
+ * cluster of 8 CTAs, while it is selected from, instead of being read back
+ * from global memory; scores[q][j < nb_q] is still written.
+ * One cluster of 8 CTAs per query, so this form pays when the batch fills the
+ * GPU (nq * 8 of at least about the SM count); with fewer queries the two
+ * separate calls spread each query over more SMs.
+ * Arguments and rules: those of qsa_index_scores and qsa_topk_blocks.  A query
+ * whose q_seq or q_pos is out of range sets the status bit and gets count 0
+ * and an all -1 selection.  When the longest possible row (min(scores_ld,
+ * max_pages_per_seq * 16) blocks) needs more shared memory per CTA than the
+ * device allows, the call enqueues the two separate kernels instead.
+ */
+QSA_API int qsa_index_topk(const qsa_cache_t* cache, const void* q_idx, const float* w, const int32_t* q_seq,
+                   const int32_t* q_pos, int32_t nq, int32_t k, float* scores, int64_t scores_ld, int32_t* sel,
+                   int32_t* count, int32_t* dev_status, void* stream);
+
+/*
+ * qsa_index_topk_smem_bytes -- host-only: the dynamic shared memory one CTA of
+ * qsa_index_topk takes for this cache group and scores_ld (about 68 KiB plus
+ * 68 B per page of the longest possible row / 8), or a negative qsa_status.
+ */
+QSA_API int qsa_index_topk_smem_bytes(const qsa_cache_t* cache, int64_t scores_ld);
+
+/*
+ * qsa_index_topk_resident_queries -- how many queries' clusters of
+ * qsa_index_topk the current device holds at once for this cache group and
+ * scores_ld (0 when a CTA's shared memory does not fit), or a negative
+ * qsa_status.  A batch of at most this many queries runs in one wave.
+ * Queries the CUDA runtime (needs a device; enqueues nothing).
+ */
+QSA_API int qsa_index_topk_resident_queries(const qsa_cache_t* cache, int64_t scores_ld);
 
 /*
  * qsa_decode_plan -- host-only helper: choose the KV chunk size for

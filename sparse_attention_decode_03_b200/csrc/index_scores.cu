@@ -11,10 +11,8 @@
 // HBM-bound stream over the side cache (256 B per block).  Each warp owns whole
 // 4 KiB kc pages (16 blocks x 128 dims): every lane issues 16-byte loads that
 // land directly in mma.sync m16n8k16 A fragments (rows = the page's 16
-// blocks, K = 128 dims, N = the 8 indexer heads).  The contraction dimension
-// is permuted consistently in A and B so that each lane reads whole 16-byte
-// chunks: lane (g, t) holds dims of chunks 4i+t (i = 0..3) of rows g and g+8.
-#include "qsa_common.cuh"
+// blocks, K = 128 dims, N = the 8 indexer heads), index_page.cuh.
+#include "index_page.cuh"
 
 namespace {
 
@@ -43,8 +41,6 @@ struct ScoreArgs {
   int32_t* st;
 };
 
-__device__ __forceinline__ float relu(float x) { return x > 0.f ? x : 0.f; }
-
 __global__ void __launch_bounds__(kWarps * 32) index_scores_kernel(ScoreArgs a) {
   pdl_launch_dependents();
   pdl_wait_previous();
@@ -69,13 +65,7 @@ __global__ void __launch_bounds__(kWarps * 32) index_scores_kernel(ScoreArgs a) 
   const int pg0 = chunk * (kWarps * ppw) + warp * ppw;
   if (pg0 >= npg) return;
 
-  // B fragments: indexer query head g, chunks 4i+t of its 128 dims.
-  uint4 qb[4];
-  const __nv_bfloat16* qrow = a.q_idx + ((size_t)q * kIdxHeads + g) * kIdxDim;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) qb[i] = ldg_nc(qrow + (4 * i + t) * 8);
-  const float w0 = a.w[q * kIdxHeads + 2 * t];
-  const float w1 = a.w[q * kIdxHeads + 2 * t + 1];
+  const IdxQuery Q = load_idx_query(a.q_idx, a.w, q);
 
   int myphys = -1;
   if (lane < ppw && pg0 + lane < npg) myphys = a.bt[(int64_t)seq * a.mpps + pg0 + lane];
@@ -90,14 +80,7 @@ __global__ void __launch_bounds__(kWarps * 32) index_scores_kernel(ScoreArgs a) 
     for (int k = 0; k < 2; ++k) {
       phys[k] = __shfl_sync(0xffffffffu, myphys, pp + k);
       ok[k] = (pg0 + pp + k < npg) && phys[k] >= 0 && phys[k] < a.num_pages;
-      if (ok[k]) {
-        const __nv_bfloat16* base = a.kc + (size_t)phys[k] * kBlocksPerPage * kIdxDim;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          ra[k][i] = ldg_stream(base + (size_t)g * kIdxDim + (4 * i + t) * 8);
-          rb[k][i] = ldg_stream(base + (size_t)(g + 8) * kIdxDim + (4 * i + t) * 8);
-        }
-      }
+      if (ok[k]) load_idx_page(a.kc, phys[k], ra[k], rb[k]);
     }
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
@@ -111,19 +94,8 @@ __global__ void __launch_bounds__(kWarps * 32) index_scores_kernel(ScoreArgs a) 
         if (t == 1 && blk_hi < nb) srow[blk_hi] = -INFINITY;
         continue;
       }
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        mma_bf16_16816(acc, ra[k][i].x, rb[k][i].x, ra[k][i].y, rb[k][i].y, qb[i].x, qb[i].y);
-        mma_bf16_16816(acc, ra[k][i].z, rb[k][i].z, ra[k][i].w, rb[k][i].w, qb[i].z, qb[i].w);
-      }
-      // acc: (block g, heads 2t, 2t+1), (block g+8, heads 2t, 2t+1)
-      float s_lo = w0 * relu(acc[0]) + w1 * relu(acc[1]);
-      float s_hi = w0 * relu(acc[2]) + w1 * relu(acc[3]);
-      s_lo += __shfl_xor_sync(0xffffffffu, s_lo, 1);
-      s_hi += __shfl_xor_sync(0xffffffffu, s_hi, 1);
-      s_lo += __shfl_xor_sync(0xffffffffu, s_lo, 2);
-      s_hi += __shfl_xor_sync(0xffffffffu, s_hi, 2);
+      float s_lo, s_hi;
+      score_idx_page(ra[k], rb[k], Q, s_lo, s_hi);
       if (t == 0 && blk_lo < nb) srow[blk_lo] = s_lo;
       if (t == 1 && blk_hi < nb) srow[blk_hi] = s_hi;
     }
@@ -134,11 +106,11 @@ __global__ void __launch_bounds__(kWarps * 32) index_scores_kernel(ScoreArgs a) 
 // Query-tiled variant for calls with many queries per sequence (chunked
 // prefill / extend): the queries of one sequence all read the same side cache,
 // so the work is a dense contraction [queries x 8 heads] x 128 x [blocks] and
-// a CTA of 16 consecutive queries reads each 128-block kc tile once for all of
+// a CTA of 32 consecutive queries reads each 128-block kc tile once for all of
 // them.  Queries of a CTA that belong to different sequences are handled by
 // one pass per distinct sequence.
 
-constexpr int kTQ = 16;                   // queries per CTA
+constexpr int kTQ = 32;                   // queries per CTA
 constexpr int kTB = 128;                  // blocks per kc tile
 constexpr int kTChunkBlocks = 8192;       // blocks per CTA (gridDim.y splits longer rows)
 
@@ -168,12 +140,12 @@ __device__ __forceinline__ void cp_async_wait_group() {
 // ---------------------------------------------------------------------------
 // The contraction runs on the 5th-generation tensor cores (tcgen05): per
 // 128-block kc tile, D[block][query*8 + head] = kc[block] .
-// q_idx[query][head] for the CTA's 16 queries, accumulated in tensor memory
-// (M = 128 blocks, N = 128, K = 128 dims in 8 steps of 16).  One TMEM lane per
+// q_idx[query][head] for the CTA's 32 queries, accumulated in tensor memory
+// (M = 128 blocks, N = 256, K = 128 dims in 8 steps of 16).  One TMEM lane per
 // block, so the w * ReLU head sum of a (query, block) score stays inside one
 // thread and the score stores are coalesced.
 //   warps 0-3  epilogue: tcgen05.ld of TMEM lanes 32w..32w+31, head sums, stores
-//   warp 4     TMEM allocation (512 columns: four accumulator buffers) and the
+//   warp 4     TMEM allocation (512 columns: two accumulator buffers) and the
 //              MMA issue (one elected thread), tcgen05.commit to mbarriers
 //   warps 5-8  producers: 16-byte cp.async of q_idx (once) and of every kc
 //              tile into the canonical K-major, no-swizzle operand layout
@@ -181,33 +153,36 @@ __device__ __forceinline__ void cp_async_wait_group() {
 //              16-element K step 128 B apart, 8-row groups 256 B apart), then
 //              a proxy fence and an mbarrier arrival per tile (a tile is
 //              published once the copies of the tile two later are issued,
-//              so three tiles are in flight per thread; 5-stage ring)
+//              so three tiles are in flight per thread; 4-stage ring)
 // All waits are bounded; on expiry the CTA records QSA_DEV_TIMEOUT, stops
 // issuing work, drains what it issued and frees its tensor memory.
 
-constexpr int kUStages = 5;
+constexpr int kUStages = 4;
 constexpr int kUTileBytes = kTB * kIdxDim * 2;                 // 32 KiB: one operand of 128 rows
 constexpr int kUEpiWarps = 4, kUMmaWarp = 4, kUProdWarp0 = 5, kUProdWarps = 4;
 constexpr int kUThreads = (kUProdWarp0 + kUProdWarps) * 32;    // 288
 constexpr int kUProdThreads = kUProdWarps * 32;
-constexpr int kUAcc = 4;                                       // accumulator buffers in tensor memory
-constexpr int kUTmemCols = kUAcc * 128;
-constexpr int kUOffB = 0;                                      // q_idx operand (128 rows)
-constexpr int kUOffA = kUOffB + kUTileBytes;                   // kc ring
-constexpr int kUOffW = kUOffA + kUStages * kUTileBytes;        // [16][8] weights
-constexpr int kUOffMeta = kUOffW + kTQ * kIdxHeads * 4;        // t_seq[16], t_nb[16], t_list[16], count, tmem, abort
+constexpr int kUN = kTQ * kIdxHeads;                           // 256: MMA N = the CTA's queries x heads
+constexpr int kUBBytes = kUN * kIdxDim * 2;                    // 64 KiB: the q_idx operand
+constexpr int kUAcc = 2;                                       // accumulator buffers in tensor memory
+constexpr int kUTmemCols = kUAcc * kUN;
+constexpr int kUOffB = 0;                                      // q_idx operand (256 rows)
+constexpr int kUOffA = kUOffB + kUBBytes;                      // kc ring
+constexpr int kUOffW = kUOffA + kUStages * kUTileBytes;        // [32][8] weights
+constexpr int kUOffMeta = kUOffW + kTQ * kIdxHeads * 4;        // t_seq[32], t_nb[32], t_list[32], count, tmem, abort
 constexpr int kUOffBar = (kUOffMeta + (3 * kTQ + 4) * 4 + 7) & ~7;
 constexpr int kUNumBars = 2 * kUStages + 2 * kUAcc + 2;        // full/empty per stage, acc full/empty, b_full, done
 constexpr int kUSmem = kUOffBar + kUNumBars * 8;
 constexpr uint32_t kUIdesc = (1u << 4)                       // D: fp32
                            | (1u << 7) | (1u << 10)          // A, B: bf16
-                           | ((uint32_t)(128 >> 3) << 17)    // N = 128
+                           | ((uint32_t)(kUN >> 3) << 17)    // N = 256
                            | ((uint32_t)(128 >> 4) << 24);   // M = 128
 constexpr uint64_t kUWaitNs = 2000000000ull;
 
-// byte offset of 16-byte chunk c (dims 8c .. 8c+7) of operand row r
+// byte offset of 16-byte chunk c (dims 8c .. 8c+7) of row r of a `rows`-row operand
+template <int rows>
 __device__ __forceinline__ uint32_t umma_off(int r, int c) {
-  return (uint32_t)((c >> 1) * 4096 + (r >> 3) * 256 + (c & 1) * 128 + (r & 7) * 16);
+  return (uint32_t)((c >> 1) * (rows * 32) + (r >> 3) * 256 + (c & 1) * 128 + (r & 7) * 16);
 }
 
 // shared-memory matrix descriptor: K-major, no swizzle, LBO 128 B, SBO 256 B
@@ -292,7 +267,7 @@ __global__ void __launch_bounds__(kUThreads, 1) index_scores_umma_kernel(TiledAr
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kUMmaWarp) {  // tensor memory for two 128 x 128 fp32 accumulators
+  if (warp == kUMmaWarp) {  // tensor memory for two 128 x 256 fp32 accumulators
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(t_tmem)),
                  "r"(kUTmemCols)
                  : "memory");
@@ -359,7 +334,7 @@ __global__ void __launch_bounds__(kUThreads, 1) index_scores_umma_kernel(TiledAr
     for (int e = pt; e < kTQ * kIdxHeads * 16; e += kUProdThreads) {
       const int r = e >> 4, c = e & 15;
       const int q = q0 + (r >> 3);
-      const uint32_t dst = sb + kUOffB + umma_off(r, c);
+      const uint32_t dst = sb + kUOffB + umma_off<kUN>(r, c);
       if (q < a.nq)
         cp_async16_cg(dst, a.q_idx + ((size_t)q * kIdxHeads + (r & 7)) * kIdxDim + c * 8);
       else
@@ -380,21 +355,24 @@ __global__ void __launch_bounds__(kUThreads, 1) index_scores_umma_kernel(TiledAr
         if (j >= kUStages && !uwait(bar_empty + stage * 8, (uint32_t)((j / kUStages - 1) & 1), abort_flag, a.st))
           break;
         const uint32_t tile = sb + kUOffA + stage * kUTileBytes;
-        // this thread's 16 chunks: chunk c = pt % 16 of rows pt / 16 + 8k; their page ids are
-        // loaded first, all together (the copies below are compiler barriers)
+        // warp w copies chunks 4w .. 4w+3 of every row; lane l takes row 8k + (l & 7),
+        // chunk 4w + (l >> 3): one warp instruction writes 8 rows x 4 chunks, which the
+        // canonical layout puts in 4 lines of 8 distinct 16-byte bank groups (the
+        // minimum 4 wavefronts for 512 B), and reads 8 x 64 contiguous bytes.  The
+        // page ids are loaded first, all together (the copies are compiler barriers).
         constexpr int kPer = kTB * 16 / kUProdThreads;  // 16
-        const int c = pt & 15;
+        const int c = 4 * (pt >> 5) + ((pt & 31) >> 3);
         int phys[kPer];
 #pragma unroll
         for (int k = 0; k < kPer; ++k) {
-          const int64_t b = b0 + (pt >> 4) + 8 * k;
+          const int64_t b = b0 + 8 * k + (pt & 7);
           phys[k] = b < B1 ? __ldg(a.bt + (int64_t)S * a.mpps + b / kBlocksPerPage) : -1;
         }
 #pragma unroll
         for (int k = 0; k < kPer; ++k) {
-          const int r = (pt >> 4) + 8 * k;
+          const int r = 8 * k + (pt & 7);
           const int64_t b = b0 + r;
-          const uint32_t dst = tile + umma_off(r, c);
+          const uint32_t dst = tile + umma_off<kTB>(r, c);
           if (b < B1 && phys[k] >= 0 && phys[k] < a.num_pages) {
             cp_async16_cg(dst, a.kc + ((size_t)phys[k] * kBlocksPerPage + b % kBlocksPerPage) * kIdxDim + c * 8);
           } else {
@@ -435,8 +413,8 @@ __global__ void __launch_bounds__(kUThreads, 1) index_scores_umma_kernel(TiledAr
           tc_fence_after();
           const uint64_t adesc0 = umma_desc(sb + kUOffA + stage * kUTileBytes);
 #pragma unroll
-          for (int ks = 0; ks < kIdxDim / 16; ++ks)  // 4096 B per 16-element K step, in 16-B units
-            umma_f16(tmem + acc * 128, adesc0 + (uint64_t)(ks * 256), bdesc0 + (uint64_t)(ks * 256), kUIdesc,
+          for (int ks = 0; ks < kIdxDim / 16; ++ks)  // per 16-element K step: rows * 32 B, in 16-B units
+            umma_f16(tmem + acc * kUN, adesc0 + (uint64_t)(ks * kTB * 2), bdesc0 + (uint64_t)(ks * kUN * 2), kUIdesc,
                      ks > 0 ? 1u : 0u);
           umma_commit(bar_empty + stage * 8);  // the kc stage is free once these MMAs finish
           umma_commit(bar_accf + acc * 8);     // the accumulator is ready
@@ -462,7 +440,7 @@ __global__ void __launch_bounds__(kUThreads, 1) index_scores_umma_kernel(TiledAr
         if (!uwait(bar_accf + acc * 8, (uint32_t)((j / kUAcc) & 1), abort_flag, a.st)) goto epi_done;
         tc_fence_after();
         float sc[kTQ];
-        const uint32_t taddr = tmem + acc * 128 + ((uint32_t)(32 * warp) << 16);
+        const uint32_t taddr = tmem + acc * kUN + ((uint32_t)(32 * warp) << 16);
 #pragma unroll
         for (int h8 = 0; h8 < kTQ / 8; ++h8) {  // 4 loads of two queries (16 columns) each, then one wait
           uint32_t r[4][16];

@@ -62,6 +62,9 @@ def _load() -> ctypes.CDLL:
         "qsa_append_kv": (ctypes.c_int, [PC, P, P, P, P, P, I32, P, P]),
         "qsa_index_scores": (ctypes.c_int, [PC, P, P, P, P, I32, P, I64, P, P]),
         "qsa_topk_blocks": (ctypes.c_int, [P, I64, P, I32, I32, P, P, P, P]),
+        "qsa_index_topk": (ctypes.c_int, [PC, P, P, P, P, I32, I32, P, I64, P, P, P, P]),
+        "qsa_index_topk_smem_bytes": (ctypes.c_int, [PC, I64]),
+        "qsa_index_topk_resident_queries": (ctypes.c_int, [PC, I64]),
         "qsa_decode_plan": (ctypes.c_int, [I32, I32, I32, I32, ctypes.POINTER(I32), ctypes.POINTER(I32)]),
         "qsa_sparse_decode": (ctypes.c_int, [PC, P, I32, I32, P, P, P, P, I32, F, I32, I32, P, P, P, P]),
         "qsa_combine": (ctypes.c_int, [P, P, I32, I32, I32, P, P, P]),
@@ -214,6 +217,47 @@ def qsa_topk_blocks(scores, q_pos, k: int, sel, count, dev_status=None, stream=N
         _req(dev_status, "dev_status", torch.int32, (1,))
     _check("qsa_topk_blocks", LIB.qsa_topk_blocks(_ptr(scores), int(scores.shape[1]), _ptr(q_pos), nq, int(k),
                                                   _ptr(sel), _ptr(count), _ptr(dev_status), _stream(stream)))
+
+
+def qsa_index_topk(cache: PagedCache, q_idx, w, q_seq, q_pos, k: int, scores, sel, count, dev_status=None,
+                   stream=None):
+    """qsa_index_scores + qsa_topk_blocks in one kernel (a cluster of 8 CTAs per
+    query keeps the score row on chip while it selects from it)."""
+    nq = int(q_seq.shape[0])
+    _req(q_idx, "q_idx", torch.bfloat16, (nq, IDX_HEADS, IDX_DIM))
+    _req(w, "w", torch.float32, (nq, IDX_HEADS))
+    _req(q_seq, "q_seq", torch.int32, (nq,))
+    _req(q_pos, "q_pos", torch.int32, (nq,))
+    _req(scores, "scores", torch.float32, (nq, None))
+    _req(sel, "sel", torch.int32, (nq, k))
+    _req(count, "count", torch.int32, (nq,))
+    if dev_status is not None:
+        _req(dev_status, "dev_status", torch.int32, (1,))
+    _check("qsa_index_topk", LIB.qsa_index_topk(ctypes.byref(cache.struct()), _ptr(q_idx), _ptr(w), _ptr(q_seq),
+                                                _ptr(q_pos), nq, int(k), _ptr(scores), int(scores.shape[1]),
+                                                _ptr(sel), _ptr(count), _ptr(dev_status), _stream(stream)))
+
+
+def index_topk_smem_bytes(cache: PagedCache, scores_ld: int) -> int:
+    r = LIB.qsa_index_topk_smem_bytes(ctypes.byref(cache.struct()), int(scores_ld))
+    _check("qsa_index_topk_smem_bytes", r if r < 0 else QSA_OK)
+    return r
+
+
+def index_topk_resident_queries(cache: PagedCache, scores_ld: int) -> int:
+    r = LIB.qsa_index_topk_resident_queries(ctypes.byref(cache.struct()), int(scores_ld))
+    _check("qsa_index_topk_resident_queries", r if r < 0 else QSA_OK)
+    return r
+
+
+def fused_selection_pays(nq: int, max_seqs: int, sms: int, resident: int) -> bool:
+    """Whether a step of nq queries should run the fused indexer + selection:
+    its 8-CTA clusters fill the GPU (nq * 8 >= the SM count) and all fit at
+    once (nq <= resident: with a second wave the longest rows start late and
+    the two-call form, which spreads a row over many CTAs, is faster), and the
+    call is decode-shaped (fewer than 8 queries per sequence on average;
+    prefill calls take the tensor-core query-tiled indexer)."""
+    return nq * 8 >= sms and nq <= resident and nq < 8 * max_seqs
 
 
 def qsa_decode_plan(nq: int, hkv: int, k: int, target_ctas: int) -> tuple[int, int]:
@@ -380,20 +424,29 @@ def bind_append_kv(cache: PagedCache, k_new, v_new, kidx_new, seq_id, pos, dev_s
 class Decoder:
     """Holds the per-step buffers (scores, selection, split partials, outputs) for
     up to `max_nq` queries and runs index_scores -> topk -> sparse_decode ->
-    combine on the current stream, with no host synchronisation."""
+    combine on the current stream, with no host synchronisation.
+
+    ``fused=True`` runs the first two as the one fused call qsa_index_topk;
+    ``fused=None`` chooses it when fused_selection_pays(max_nq, ...)."""
 
     def __init__(self, cache: PagedCache, hq: int, max_nq: int, k: int = 512, scale: float = 1.0 / 16.0,
-                 target_ctas: int | None = None, chunk_units: int | None = None, scores_ld: int | None = None):
+                 target_ctas: int | None = None, chunk_units: int | None = None, scores_ld: int | None = None,
+                 fused: bool | None = False):
         dev = cache.device
         self.cache, self.hq, self.k, self.scale, self.max_nq = cache, hq, k, scale, max_nq
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
         if target_ctas is None:
-            target_ctas = torch.cuda.get_device_properties(dev).multi_processor_count
+            target_ctas = sms
+        self.scores_ld = scores_ld or cache.max_pages_per_seq * BLOCKS_PER_PAGE
+        if fused is None:
+            fused = (cache.kc_pages is not None and fused_selection_pays(
+                max_nq, cache.max_seqs, sms, index_topk_resident_queries(cache, self.scores_ld)))
+        self.fused = bool(fused)
         if chunk_units is None:
             chunk_units, self.max_splits = qsa_decode_plan(max_nq, cache.num_kv_heads, k, target_ctas)
         else:
             self.max_splits = splits_bound(k, chunk_units)
         self.chunk_units = chunk_units
-        self.scores_ld = scores_ld or cache.max_pages_per_seq * BLOCKS_PER_PAGE
         self.scores = torch.empty((max_nq, self.scores_ld), dtype=torch.float32, device=dev)
         self.sel = torch.empty((max_nq, k), dtype=torch.int32, device=dev)
         self.count = torch.empty((max_nq,), dtype=torch.int32, device=dev)
@@ -407,8 +460,9 @@ class Decoder:
         self.dev_status = torch.zeros((1,), dtype=torch.int32, device=dev)
 
     def bind(self, q, q_idx, w, q_seq, q_pos, stream=None) -> list:
-        """Validate the step inputs once and return the four pre-bound launches
-        (index_scores, topk, sparse_decode, combine) for them."""
+        """Validate the step inputs once and return the pre-bound launches for
+        them: (index_scores, topk, sparse_decode, combine), or (index_topk,
+        sparse_decode, combine) when fused."""
         nq = int(q_seq.shape[0])
         assert nq <= self.max_nq
         hq = self.hq
@@ -423,11 +477,17 @@ class Decoder:
         st = self.cache.struct()
         ds, sp = _ptr(self.dev_status), _stream(stream)
         keep = (self.cache, st, q, q_idx, w, q_seq, q_pos, self.dev_status)
-        return [
-            BoundCall("qsa_index_scores", (ctypes.byref(st), _ptr(q_idx), _ptr(w), _ptr(q_seq), _ptr(q_pos), nq,
-                                           _ptr(sc), int(sc.shape[1]), ds, sp), keep),
-            BoundCall("qsa_topk_blocks", (_ptr(sc), int(sc.shape[1]), _ptr(q_pos), nq, self.k, _ptr(se), _ptr(cn),
-                                          ds, sp), keep),
+        if self.fused:
+            select = [BoundCall("qsa_index_topk", (ctypes.byref(st), _ptr(q_idx), _ptr(w), _ptr(q_seq), _ptr(q_pos),
+                                                   nq, self.k, _ptr(sc), int(sc.shape[1]), _ptr(se), _ptr(cn), ds,
+                                                   sp), keep)]
+        else:
+            select = [
+                BoundCall("qsa_index_scores", (ctypes.byref(st), _ptr(q_idx), _ptr(w), _ptr(q_seq), _ptr(q_pos), nq,
+                                               _ptr(sc), int(sc.shape[1]), ds, sp), keep),
+                BoundCall("qsa_topk_blocks", (_ptr(sc), int(sc.shape[1]), _ptr(q_pos), nq, self.k, _ptr(se),
+                                              _ptr(cn), ds, sp), keep)]
+        return select + [
             BoundCall("qsa_sparse_decode", (ctypes.byref(st), _ptr(q), nq, hq, _ptr(q_seq), _ptr(q_pos), _ptr(se),
                                             _ptr(cn), self.k, float(self.scale), self.chunk_units, self.max_splits,
                                             _ptr(po), _ptr(pl), ds, sp), keep),
@@ -460,8 +520,11 @@ class Decoder:
         assert nq <= self.max_nq
         sc, se, cn = self.scores[:nq], self.sel[:nq], self.count[:nq]
         po, pl = self.part_o[:nq], self.part_lse[:nq]
-        qsa_index_scores(self.cache, q_idx, w, q_seq, q_pos, sc, self.dev_status, stream)
-        qsa_topk_blocks(sc, q_pos, self.k, se, cn, self.dev_status, stream)
+        if self.fused:
+            qsa_index_topk(self.cache, q_idx, w, q_seq, q_pos, self.k, sc, se, cn, self.dev_status, stream)
+        else:
+            qsa_index_scores(self.cache, q_idx, w, q_seq, q_pos, sc, self.dev_status, stream)
+            qsa_topk_blocks(sc, q_pos, self.k, se, cn, self.dev_status, stream)
         qsa_sparse_decode(self.cache, q, q_seq, q_pos, se, cn, self.k, self.scale, self.chunk_units,
                           self.max_splits, po, pl, self.dev_status, stream)
         qsa_combine(po, pl, self.out[:nq], self.lse[:nq], stream)

@@ -25,7 +25,7 @@ def test_library_exports_every_declared_symbol():
     lib = ctypes.CDLL(qsa.LIB_PATH)
     for n in header_functions():
         assert hasattr(lib, n), n
-    assert qsa.ABI_VERSION == 4
+    assert qsa.ABI_VERSION == 5
     assert qsa.status_string(0) == "QSA_OK" and qsa.status_string(-3) == "QSA_ERR_CUDA"
 
 
@@ -85,6 +85,22 @@ def test_host_validation_returns_before_any_cuda_call():
     kc_only = qsa.qsa.qsa_cache_t(None, 0x1000, 0x1000, 0x1000, 10, 2, 4, 2)
     assert L.qsa_sparse_decode(ctypes.byref(kc_only), fake, 1, 16, fake, fake, fake, fake, 16, 0.0625, 16, 4, fake,
                                fake, None, None) == -1
+    # fused indexer + selection: the checks of both separate calls
+    assert L.qsa_index_topk(cp, fake, fake, fake, fake, 1, 4096, fake, 16, fake, fake, None, None) == -1
+    assert L.qsa_index_topk(cp, fake, fake, fake, fake, 1, 16, fake, 0, fake, fake, None, None) == -1
+    assert L.qsa_index_topk(cp, fake, fake, fake, fake, 1, 16, fake, 16, None, fake, None, None) == -1
+    assert L.qsa_index_topk(cp, ctypes.c_void_p(0x1008), fake, fake, fake, 1, 16, fake, 16, fake, fake, None,
+                            None) == -1
+    assert L.qsa_index_topk(ctypes.byref(kv_only), fake, fake, fake, fake, 1, 16, fake, 16, fake, fake, None,
+                            None) == -1
+    assert L.qsa_index_topk(cp, fake, fake, fake, fake, 0, 16, fake, 16, fake, fake, None, None) == 0
+    # its shared memory: a fixed part plus 68 B (page id + 16 score keys) per page of a CTA's eighth of the row
+    wide = qsa.qsa.qsa_cache_t(0x1000, 0x1000, 0x1000, 0x1000, 10, 2, 4096, 2)
+    wp = ctypes.byref(wide)
+    b_long, b_short = L.qsa_index_topk_smem_bytes(wp, 65536), L.qsa_index_topk_smem_bytes(wp, 1024)
+    assert b_long - b_short == (512 - 8) * 68 and 64 << 10 < b_short < 72 << 10
+    assert L.qsa_index_topk_smem_bytes(wp, 1 << 30) == L.qsa_index_topk_smem_bytes(wp, 65536)  # capped by the table
+    assert L.qsa_index_topk_smem_bytes(wp, 0) == -1
     # K/V storage types: BF16 and FP8 e4m3 only
     bad = qsa.qsa.qsa_cache_t(0x1000, 0x1000, 0x1000, 0x1000, 10, 2, 4, 2, 7)
     bp = ctypes.byref(bad)

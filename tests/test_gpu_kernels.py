@@ -169,13 +169,13 @@ def test_index_scores_and_topk_bit_exact(name, lengths, k):
 
 @pytest.mark.parametrize("lengths,new,k", [
     ([700, 2900, 33], 37, 64),     # 111 queries: ragged last tile, tiles spanning two sequences
-    ([36000], 20, 512),            # rows longer than one CTA's 8,192-block chunk
+    ([36000], 40, 512),            # rows longer than one CTA's 8,192-block chunk, ragged tile
 ])
 def test_query_tiled_index_scores_bit_exact(lengths, new, k):
     """Chunked-prefill calls (many queries per sequence) take the query-tiled
     indexer; its scores and the selections must match the oracle exactly."""
     wl = C.shrink(C.get("prefill"), lengths, new_tokens=new, page_perm=True, k_top=k)
-    assert wl.nq >= 8 * wl.batch and wl.nq >= 16
+    assert wl.nq >= 8 * wl.batch and wl.nq >= 32
     cache, dec, st = run_step(wl, k=k)
     assert st == 0
     sc = dec.scores.cpu().numpy()
