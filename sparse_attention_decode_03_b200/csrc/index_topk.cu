@@ -106,7 +106,9 @@ __device__ __forceinline__ void st_cluster(void* p, uint32_t rank, uint32_t v) {
 }
 
 __global__ void __launch_bounds__(kFThreads, 2) index_topk_kernel(FusedArgs a) {
-  pdl_launch_dependents();
+  // The next kernel is allowed to launch only once every cluster has reached
+  // its selection (or left): launched earlier, its CTAs would take the shared
+  // memory this grid's later clusters need and push them into a second wave.
   pdl_wait_previous();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   FSmem& S = *reinterpret_cast<FSmem*>(smem_raw);
@@ -272,6 +274,7 @@ __global__ void __launch_bounds__(kFThreads, 2) index_topk_kernel(FusedArgs a) {
     if (tid == 0) st_cluster(&S.wcnt[rank], 0u, over ? (uint32_t)kFList + 1 : total);
   }
   cluster_barrier();  // 2: the leader holds every CTA's list; no shared memory is touched remotely after this
+  pdl_launch_dependents();
   if (!leader) return;
 
   // ---------------- B3. the exact select on the leader (warp w: the list of CTA w)

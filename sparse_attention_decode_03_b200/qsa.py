@@ -426,12 +426,13 @@ class Decoder:
     up to `max_nq` queries and runs index_scores -> topk -> sparse_decode ->
     combine on the current stream, with no host synchronisation.
 
-    ``fused=True`` runs the first two as the one fused call qsa_index_topk;
-    ``fused=None`` chooses it when fused_selection_pays(max_nq, ...)."""
+    ``fused=True`` runs the first two as the one fused call qsa_index_topk,
+    ``fused=False`` as the two calls; the default chooses the fused call when
+    fused_selection_pays(max_nq, ...)."""
 
     def __init__(self, cache: PagedCache, hq: int, max_nq: int, k: int = 512, scale: float = 1.0 / 16.0,
                  target_ctas: int | None = None, chunk_units: int | None = None, scores_ld: int | None = None,
-                 fused: bool | None = False):
+                 fused: bool | None = None):
         dev = cache.device
         self.cache, self.hq, self.k, self.scale, self.max_nq = cache, hq, k, scale, max_nq
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
