@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--context", type=int, default=0, help="override every context length (profiling a small case)")
     ap.add_argument("--select", choices=["auto", "fused", "split"], default="auto",
                     help="indexer + top-K as one fused kernel, as two kernels, or as the library chooses")
+    ap.add_argument("--merge", choices=["kernel", "separate"], default="separate",
+                    help="split-KV merge inside the attention kernel, or as the separate combine kernel")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time budget for the CPU baseline")
     ap.add_argument("--dcp", type=int, default=0,
@@ -193,8 +195,9 @@ def algorithmic_bytes(wl: C.Workload, count: np.ndarray, q_pos: np.ndarray, spli
     out = wl.nq * wl.hq * 256 * 2
     combine = partials + out
     index_topk = index + wl.nq * wl.k_top * 4  # the fused kernel never reads the scores back
+    attention = decode + out                   # split kernel + its in-kernel merge
     return {"append_kv": append, "index_scores": index, "topk": topk, "index_topk": index_topk,
-            "sparse_decode": decode, "combine": combine,
+            "sparse_decode": decode, "combine": combine, "sparse_attention": attention,
             "pipeline_spec": side + kv + out, "side_cache": side, "selected_kv": kv, "output": out}
 
 
@@ -209,8 +212,9 @@ def measured_peaks():
 def kernel_source_sha(kernel: str) -> str:
     """Hash of the kernel's source file and of every shared device header."""
     csrc = os.path.join(ROOT, "sparse_attention_decode_03_b200", "csrc")
+    src = {"sparse_attention": "sparse_decode", "topk": "topk", "append_kv": "append_kv"}.get(kernel, kernel)
     h = hashlib.sha256()
-    for f in [os.path.join(csrc, f"{kernel}.cu")] + sorted(glob.glob(os.path.join(csrc, "*.cuh"))):
+    for f in [os.path.join(csrc, f"{src}.cu")] + sorted(glob.glob(os.path.join(csrc, "*.cuh"))):
         if os.path.exists(f):
             h.update(open(f, "rb").read())
     return h.hexdigest()[:16]
@@ -314,14 +318,16 @@ def run_native(args, rank, ws, local):
     torch.cuda.synchronize()
     inp = io.dev
     dec = qsa.Decoder(cache, wl.hq, wl.nq, k=wl.k_top, scale=wl.scale, target_ctas=sms,
-                      chunk_units=H.chunk_units_for(wl), fused={"auto": None, "fused": True, "split": False}[args.select])
+                      chunk_units=H.chunk_units_for(wl), fused={"auto": None, "fused": True, "split": False}[args.select],
+                      merged=args.merge == "kernel")
     dec.dev_status = st
     saved_partial = cache.kc_partial.clone()
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     flush_read = torch.ones(64 << 20, dtype=torch.int32, device=dev)
     flush_sink = torch.zeros((), dtype=torch.int64, device=dev)
     stream = torch.cuda.Stream(device=dev)   # the step's stream (captured into a CUDA graph below)
-    names = ["append_kv"] + (["index_topk"] if dec.fused else ["index_scores", "topk"]) + ["sparse_decode", "combine"]
+    names = (["append_kv"] + (["index_topk"] if dec.fused else ["index_scores", "topk"])
+             + (["sparse_attention"] if dec.merged else ["sparse_decode", "combine"]))
 
     calls = [qsa.bind_append_kv(cache, inp["k_new"], inp["v_new"], inp["kidx_new"], inp["seq_id"], inp["pos"], st,
                                 stream=stream)]
@@ -439,8 +445,8 @@ def run_native(args, rank, ws, local):
         raise RuntimeError(f"device status after the e2e steps: {qsa.dev_status_names(status)}")
     e2e_total = max_over_ranks(sum(e2e_ms), ws)
     e2e_value = ws * wl.nq * len(e2e_ms) / (e2e_total / 1000.0)
-    # append scatter + append partial + (scores + top-K, or the fused kernel) + attention + combine
-    launches_per_step = 5 if dec.fused else 6
+    # append scatter + append partial + (scores + top-K, or the fused kernel) + (attention + combine, or merged)
+    launches_per_step = 2 + (1 if dec.fused else 2) + (1 if dec.merged else 2)
 
     # ---- roofline of the dominant kernel
     count = dec.count[:wl.nq].cpu().numpy()
@@ -463,8 +469,9 @@ def run_native(args, rank, ws, local):
         "warmup": args.warmup, "ms_per_step": mean_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "e4m3 kv + bf16" if wl.kv_fp8 else "bf16", "data": "synthetic",
         "config": {**wl.describe(), "l2": "flushed between timed steps (512 MiB write, then 256 MiB read); inputs also larger than L2",
-                   "step": ("append_kv + index_topk (fused) + sparse_decode + combine, one CUDA graph" if dec.fused
-                            else "append_kv + index_scores + topk_blocks + sparse_decode + combine, one CUDA graph"),
+                   "step": " + ".join(["append_kv"] + (["index_topk (fused)"] if dec.fused else ["index_scores", "topk_blocks"])
+                                      + (["sparse_attention (split kernel with in-kernel merge)"] if dec.merged
+                                         else ["sparse_decode", "combine"])) + ", one CUDA graph",
                    "kernel_timing": "per kernel: CUDA events around a graph of 8 x (L2 flush, kernel) minus one of 8 x (L2 flush), / 8",
                    "parallelism": f"dp{ws} (independent replicas)" if ws > 1 else "single GPU",
                    "chunk_units": dec.chunk_units, "max_splits": dec.max_splits},

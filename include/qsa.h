@@ -132,7 +132,7 @@ QSA_API const char* qsa_status_string(int status);
 
 /* ABI version of this header (bumped on any signature change). */
 QSA_API int qsa_abi_version(void);
-#define QSA_ABI_VERSION 5
+#define QSA_ABI_VERSION 6
 
 /*
  * qsa_append_kv -- write n new tokens into the cache group.
@@ -259,6 +259,25 @@ QSA_API int qsa_sparse_decode(const qsa_cache_t* cache, const void* q, int32_t n
                       const int32_t* q_pos, const int32_t* sel, const int32_t* count, int32_t k, float scale,
                       int32_t chunk_units, int32_t max_splits, float* part_o, float* part_lse,
                       int32_t* dev_status, void* stream);
+
+/*
+ * qsa_sparse_attention -- qsa_sparse_decode followed by qsa_combine in one
+ * kernel ([DCP]: the split results are combined afterwards; here the combine
+ * runs inside the split kernel).  Every CTA writes its split partials exactly
+ * as qsa_sparse_decode does; the CTA that writes the last split of a (query,
+ * KV head) pair -- counted with a device-scope atomic in pair_done -- merges
+ * that pair's splits into out / lse with qsa_combine's arithmetic, so out and
+ * lse equal those of the two calls bit for bit.
+ *   pair_done int32 [nq][Hkv], all zero on entry; the call leaves it all zero
+ *             (after a QSA_DEV_TIMEOUT status the caller must zero it again)
+ *   out bf16 [nq][hq][256] (8-byte aligned); lse fp32 [nq][hq]
+ * Other arguments, rules and errors: those of qsa_sparse_decode.
+ */
+QSA_API int qsa_sparse_attention(const qsa_cache_t* cache, const void* q, int32_t nq, int32_t hq,
+                         const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel, const int32_t* count,
+                         int32_t k, float scale, int32_t chunk_units, int32_t max_splits, float* part_o,
+                         float* part_lse, int32_t* pair_done, void* out, float* lse, int32_t* dev_status,
+                         void* stream);
 
 /*
  * qsa_combine -- log-sum-exp merge of the splits ([DCP]: attention results of

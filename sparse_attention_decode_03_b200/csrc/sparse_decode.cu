@@ -137,6 +137,11 @@ struct DecodeArgs {
   int32_t max_splits;
   float* part_o;
   float* part_lse;
+  // in-kernel merge (all three null: partials only): per (query, KV group) the
+  // number of its splits written so far, zero on entry and on exit
+  int32_t* pair_done;
+  __nv_bfloat16* out;  // [nq][hq][256]
+  float* lse;          // [nq][hq]
   int32_t* st;
 };
 
@@ -429,6 +434,48 @@ __device__ __forceinline__ bool consumer_wait(const DecodeArgs& a, uint32_t bar,
         return false;
       }
     }
+  }
+}
+
+// Log-sum-exp merge of the nspl splits of pair (q, g) into out / lse, by the
+// 256 consumer threads of the CTA that wrote the pair's last split: thread t
+// owns dims 4 (t % 64) .. + 3 of rows t / 64, t / 64 + 4, ... of the group.
+// The arithmetic is that of qsa_combine (same order over the splits), so the
+// result is the same bit for bit.  Partials of other CTAs are read from L2.
+__device__ __forceinline__ void merge_pair(const DecodeArgs& a, int q, int g, int nspl, int tid) {
+  const int G = a.G;
+  const int c4 = tid & 63;
+  for (int r = tid >> 6; r < G; r += kConsumerThreads / 64) {
+    const int h = g * G + r;
+    const float* pl = a.part_lse + (size_t)q * a.max_splits * a.hq + h;
+    const float* po = a.part_o + ((size_t)q * a.max_splits * a.hq + h) * kHeadDim + 4 * c4;
+    float M = -INFINITY;
+    for (int sp = 0; sp < nspl; ++sp) M = fmaxf(M, __ldcg(pl + (size_t)sp * a.hq));
+    float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+    float lse_v = -INFINITY;
+    if (M != -INFINITY) {  // else every split is empty: zero output, lse = -inf
+      float L = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int sp = 0; sp < nspl; ++sp) {
+        const float v = __ldcg(pl + (size_t)sp * a.hq);
+        if (v == -INFINITY) continue;
+        const float e = expf(v - M);
+        const float4 x = __ldcg(reinterpret_cast<const float4*>(po + (size_t)sp * a.hq * kHeadDim));
+        L += e;
+        acc.x += e * x.x;
+        acc.y += e * x.y;
+        acc.z += e * x.z;
+        acc.w += e * x.w;
+      }
+      const float inv = 1.f / L;
+      res = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+      lse_v = M + logf(L);
+    }
+    uint2 o;
+    o.x = pack_bf16(res.x, res.y);
+    o.y = pack_bf16(res.z, res.w);
+    reinterpret_cast<uint2*>(a.out + ((size_t)q * a.hq + h) * kHeadDim)[c4] = o;
+    if (c4 == 0) a.lse[(size_t)q * a.hq + h] = lse_v;
   }
 }
 
@@ -758,6 +805,27 @@ __device__ void consumers(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_
         for (int row = tid; row < G; row += kConsumerThreads) a.part_lse[r0 + row] = -INFINITY;
       }
     }
+    if (a.pair_done) {
+      // The CTA that writes a pair's last split merges the pair: every writer
+      // fences its partial stores, one thread counts the split (device-scope
+      // atomic) and fences again before the merge reads the other splits.
+      __threadfence();
+      named_bar_sync(kBarConsumers, kConsumerThreads);
+      volatile int* last_flag = reinterpret_cast<volatile int*>(ml);  // ml is free until the next segment ends
+      const int64_t base = pair * n_slots;
+      const int nspl = (int)((base + n_slots - 1) / a.chunk - base / a.chunk) + 1;
+      if (tid == 0) {
+        const int done = atomicAdd(a.pair_done + pair, 1);
+        const bool last = done == nspl - 1;
+        if (last) a.pair_done[pair] = 0;  // every other split has counted: ready for the next call
+        __threadfence();
+        *last_flag = last ? 1 : 0;
+      }
+      named_bar_sync(kBarConsumers, kConsumerThreads);
+      const bool last = *last_flag != 0;
+      named_bar_sync(kBarConsumers, kConsumerThreads);  // the flag is read before ml is written again
+      if (last) merge_pair(a, s.q, s.g, nspl, tid);
+    }
   }
 }
 
@@ -809,11 +877,12 @@ int launch_decode(const DecodeArgs& a, int64_t grid, void* stream) {
 
 int32_t qsa_splits_bound(int32_t k, int32_t chunk);
 
-extern "C" int qsa_sparse_decode(const qsa_cache_t* cache, const void* q, int32_t nq, int32_t hq,
-                                 const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel,
-                                 const int32_t* count, int32_t k, float scale, int32_t chunk_units,
-                                 int32_t max_splits, float* part_o, float* part_lse, int32_t* dev_status,
-                                 void* stream) {
+namespace {
+
+int decode_call(const qsa_cache_t* cache, const void* q, int32_t nq, int32_t hq, const int32_t* q_seq,
+                const int32_t* q_pos, const int32_t* sel, const int32_t* count, int32_t k, float scale,
+                int32_t chunk_units, int32_t max_splits, float* part_o, float* part_lse, int32_t* pair_done,
+                void* out, float* lse, int32_t* dev_status, void* stream) {
   if (!cache || nq < 0 || hq < 1 || k < 0 || k > QSA_MAX_TOPK || chunk_units < 1 || max_splits < 1)
     return QSA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !(scale < 3.0e38f)) return QSA_ERR_INVALID_ARG;
@@ -851,8 +920,33 @@ extern "C" int qsa_sparse_decode(const qsa_cache_t* cache, const void* q, int32_
   a.max_splits = max_splits;
   a.part_o = part_o;
   a.part_lse = part_lse;
+  a.pair_done = pair_done;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.lse = lse;
   a.st = dev_status;
   const int64_t grid = (a.total_slots + a.chunk - 1) / a.chunk;
   if (grid > 0x7fffffff) return QSA_ERR_UNSUPPORTED;
   return c.kv_dtype == QSA_KV_FP8_E4M3 ? launch_decode<true>(a, grid, stream) : launch_decode<false>(a, grid, stream);
+}
+
+}  // namespace
+
+extern "C" int qsa_sparse_decode(const qsa_cache_t* cache, const void* q, int32_t nq, int32_t hq,
+                                 const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel,
+                                 const int32_t* count, int32_t k, float scale, int32_t chunk_units,
+                                 int32_t max_splits, float* part_o, float* part_lse, int32_t* dev_status,
+                                 void* stream) {
+  return decode_call(cache, q, nq, hq, q_seq, q_pos, sel, count, k, scale, chunk_units, max_splits, part_o, part_lse,
+                     nullptr, nullptr, nullptr, dev_status, stream);
+}
+
+extern "C" int qsa_sparse_attention(const qsa_cache_t* cache, const void* q, int32_t nq, int32_t hq,
+                                    const int32_t* q_seq, const int32_t* q_pos, const int32_t* sel,
+                                    const int32_t* count, int32_t k, float scale, int32_t chunk_units,
+                                    int32_t max_splits, float* part_o, float* part_lse, int32_t* pair_done,
+                                    void* out, float* lse, int32_t* dev_status, void* stream) {
+  if (nq > 0 && (!pair_done || !out || !lse)) return QSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(out) & 7u) return QSA_ERR_INVALID_ARG;
+  return decode_call(cache, q, nq, hq, q_seq, q_pos, sel, count, k, scale, chunk_units, max_splits, part_o, part_lse,
+                     pair_done, out, lse, dev_status, stream);
 }

@@ -67,6 +67,7 @@ def _load() -> ctypes.CDLL:
         "qsa_index_topk_resident_queries": (ctypes.c_int, [PC, I64]),
         "qsa_decode_plan": (ctypes.c_int, [I32, I32, I32, I32, ctypes.POINTER(I32), ctypes.POINTER(I32)]),
         "qsa_sparse_decode": (ctypes.c_int, [PC, P, I32, I32, P, P, P, P, I32, F, I32, I32, P, P, P, P]),
+        "qsa_sparse_attention": (ctypes.c_int, [PC, P, I32, I32, P, P, P, P, I32, F, I32, I32, P, P, P, P, P, P, P]),
         "qsa_combine": (ctypes.c_int, [P, P, I32, I32, I32, P, P, P]),
         "qsa_combine_strided": (ctypes.c_int, [P, P, I32, I32, I32, I64, I64, I64, I64, P, I32, P, P]),
         "qsa_dcp_localize_tokens": (ctypes.c_int, [P, P, I32, I32, I32, I32, P, P, P]),
@@ -286,6 +287,31 @@ def qsa_sparse_decode(cache: PagedCache, q, q_seq, q_pos, sel, count, k: int, sc
         _stream(stream)))
 
 
+def qsa_sparse_attention(cache: PagedCache, q, q_seq, q_pos, sel, count, k: int, scale: float, chunk_units: int,
+                         max_splits: int, part_o, part_lse, pair_done, out, lse, dev_status=None, stream=None):
+    """qsa_sparse_decode + qsa_combine in one kernel: the CTA that writes a
+    (query, KV head) pair's last split merges it.  pair_done (int32 [nq][Hkv])
+    must be zero on entry and is zero again afterwards."""
+    nq = int(q_seq.shape[0])
+    hq = int(q.shape[1]) if q.dim() == 3 else -1
+    _req(q, "q", torch.bfloat16, (nq, hq, HEAD_DIM))
+    _req(q_seq, "q_seq", torch.int32, (nq,))
+    _req(q_pos, "q_pos", torch.int32, (nq,))
+    _req(sel, "sel", torch.int32, (nq, k))
+    _req(count, "count", torch.int32, (nq,))
+    _req(part_o, "part_o", torch.float32, (nq, max_splits, hq, HEAD_DIM))
+    _req(part_lse, "part_lse", torch.float32, (nq, max_splits, hq))
+    _req(pair_done, "pair_done", torch.int32, (nq * cache.num_kv_heads,))
+    _req(out, "out", torch.bfloat16, (nq, hq, HEAD_DIM))
+    _req(lse, "lse", torch.float32, (nq, hq))
+    if dev_status is not None:
+        _req(dev_status, "dev_status", torch.int32, (1,))
+    _check("qsa_sparse_attention", LIB.qsa_sparse_attention(
+        ctypes.byref(cache.struct()), _ptr(q), nq, hq, _ptr(q_seq), _ptr(q_pos), _ptr(sel), _ptr(count), int(k),
+        float(scale), int(chunk_units), int(max_splits), _ptr(part_o), _ptr(part_lse), _ptr(pair_done), _ptr(out),
+        _ptr(lse), _ptr(dev_status), _stream(stream)))
+
+
 def qsa_combine(part_o, part_lse, out, lse, stream=None):
     nq, S, hq = (int(x) for x in part_lse.shape)
     _req(part_o, "part_o", torch.float32, (nq, S, hq, HEAD_DIM))
@@ -428,11 +454,15 @@ class Decoder:
 
     ``fused=True`` runs the first two as the one fused call qsa_index_topk,
     ``fused=False`` as the two calls; the default chooses the fused call when
-    fused_selection_pays(max_nq, ...)."""
+    fused_selection_pays(max_nq, ...).  ``merged=True`` runs the last two as
+    the one call qsa_sparse_attention (the split kernel merges each pair's
+    splits itself), the default ``merged=False`` as qsa_sparse_decode +
+    qsa_combine (faster on B200: the merge's fences and L2 round trips in the
+    split kernel cost more than the separate launch)."""
 
     def __init__(self, cache: PagedCache, hq: int, max_nq: int, k: int = 512, scale: float = 1.0 / 16.0,
                  target_ctas: int | None = None, chunk_units: int | None = None, scores_ld: int | None = None,
-                 fused: bool | None = None):
+                 fused: bool | None = None, merged: bool = False):
         dev = cache.device
         self.cache, self.hq, self.k, self.scale, self.max_nq = cache, hq, k, scale, max_nq
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
@@ -458,6 +488,8 @@ class Decoder:
         self._out_arena = torch.empty(_align(out_bytes) + max_nq * hq * 4, dtype=torch.uint8, device=dev)
         self.out = self._out_arena[:out_bytes].view(torch.bfloat16).view(max_nq, hq, HEAD_DIM)
         self.lse = self._out_arena[_align(out_bytes):].view(torch.float32).view(max_nq, hq)
+        self.merged = bool(merged)
+        self.pair_done = torch.zeros((max_nq * cache.num_kv_heads,), dtype=torch.int32, device=dev)
         self.dev_status = torch.zeros((1,), dtype=torch.int32, device=dev)
 
     def bind(self, q, q_idx, w, q_seq, q_pos, stream=None) -> list:
@@ -488,6 +520,12 @@ class Decoder:
                                                _ptr(sc), int(sc.shape[1]), ds, sp), keep),
                 BoundCall("qsa_topk_blocks", (_ptr(sc), int(sc.shape[1]), _ptr(q_pos), nq, self.k, _ptr(se),
                                               _ptr(cn), ds, sp), keep)]
+        if self.merged:
+            return select + [
+                BoundCall("qsa_sparse_attention", (ctypes.byref(st), _ptr(q), nq, hq, _ptr(q_seq), _ptr(q_pos),
+                                                   _ptr(se), _ptr(cn), self.k, float(self.scale), self.chunk_units,
+                                                   self.max_splits, _ptr(po), _ptr(pl), _ptr(self.pair_done),
+                                                   _ptr(out), _ptr(lse), ds, sp), keep + (self.pair_done,))]
         return select + [
             BoundCall("qsa_sparse_decode", (ctypes.byref(st), _ptr(q), nq, hq, _ptr(q_seq), _ptr(q_pos), _ptr(se),
                                             _ptr(cn), self.k, float(self.scale), self.chunk_units, self.max_splits,
@@ -526,9 +564,14 @@ class Decoder:
         else:
             qsa_index_scores(self.cache, q_idx, w, q_seq, q_pos, sc, self.dev_status, stream)
             qsa_topk_blocks(sc, q_pos, self.k, se, cn, self.dev_status, stream)
-        qsa_sparse_decode(self.cache, q, q_seq, q_pos, se, cn, self.k, self.scale, self.chunk_units,
-                          self.max_splits, po, pl, self.dev_status, stream)
-        qsa_combine(po, pl, self.out[:nq], self.lse[:nq], stream)
+        if self.merged:
+            qsa_sparse_attention(self.cache, q, q_seq, q_pos, se, cn, self.k, self.scale, self.chunk_units,
+                                 self.max_splits, po, pl, self.pair_done[:nq * self.cache.num_kv_heads],
+                                 self.out[:nq], self.lse[:nq], self.dev_status, stream)
+        else:
+            qsa_sparse_decode(self.cache, q, q_seq, q_pos, se, cn, self.k, self.scale, self.chunk_units,
+                              self.max_splits, po, pl, self.dev_status, stream)
+            qsa_combine(po, pl, self.out[:nq], self.lse[:nq], stream)
         return self.out[:nq], self.lse[:nq]
 
 

@@ -25,7 +25,7 @@ def test_library_exports_every_declared_symbol():
     lib = ctypes.CDLL(qsa.LIB_PATH)
     for n in header_functions():
         assert hasattr(lib, n), n
-    assert qsa.ABI_VERSION == 5
+    assert qsa.ABI_VERSION == 6
     assert qsa.status_string(0) == "QSA_OK" and qsa.status_string(-3) == "QSA_ERR_CUDA"
 
 
@@ -85,6 +85,15 @@ def test_host_validation_returns_before_any_cuda_call():
     kc_only = qsa.qsa.qsa_cache_t(None, 0x1000, 0x1000, 0x1000, 10, 2, 4, 2)
     assert L.qsa_sparse_decode(ctypes.byref(kc_only), fake, 1, 16, fake, fake, fake, fake, 16, 0.0625, 16, 4, fake,
                                fake, None, None) == -1
+    # attention with the in-kernel merge: the decode checks plus its own buffers
+    m_args = lambda nq, pd, out: (cp, fake, nq, 16, fake, fake, fake, fake, 16, 0.0625, 16, 4, fake, fake, pd, out, fake,
+                                  None, None)
+    assert L.qsa_sparse_attention(*m_args(1, None, fake)) == -1
+    assert L.qsa_sparse_attention(*m_args(1, fake, None)) == -1
+    assert L.qsa_sparse_attention(*m_args(1, fake, ctypes.c_void_p(0x1004))) == -1   # out not 8-byte aligned
+    assert L.qsa_sparse_attention(*m_args(0, None, None)) == 0
+    assert L.qsa_sparse_attention(cp, fake, 1, 3, fake, fake, fake, fake, 16, 0.0625, 16, 4, fake, fake, fake, fake,
+                                  fake, None, None) == -1                            # Hq not a multiple of Hkv
     # fused indexer + selection: the checks of both separate calls
     assert L.qsa_index_topk(cp, fake, fake, fake, fake, 1, 4096, fake, 16, fake, fake, None, None) == -1
     assert L.qsa_index_topk(cp, fake, fake, fake, fake, 1, 16, fake, 0, fake, fake, None, None) == -1
