@@ -5,9 +5,11 @@
     python bench.py --impl reference ...   # the CPU oracle, timed on the host
 
 One step = one pass of the whole hot path over one batch: qsa_append_kv of the
-batch's new tokens (the current token of every sequence), qsa_index_scores,
-qsa_topk_blocks, qsa_sparse_decode, qsa_combine, all enqueued on one stream
-with the cache resident in HBM.  Between timed steps the open micro-block sums
+batch's new tokens (the current token of every sequence), the indexer scores
+and top-K selection (qsa_index_scores + qsa_topk_blocks, or the fused
+qsa_index_topk, as the Decoder chooses or --select forces), qsa_sparse_decode
+and qsa_combine (or the merged qsa_sparse_attention with --merge kernel), all
+enqueued on one stream with the cache resident in HBM.  Between timed steps the open micro-block sums
 are restored (the step appends the same token again) and L2 is flushed by
 writing a 512 MiB buffer; neither is inside the timed events.
 
