@@ -649,6 +649,71 @@ class StepGraph:
         return [self.events[k].elapsed_time(self.events[k + 1]) for k in range(len(self.calls))]
 
 
+class StepPipeline:
+    """Serving-style double buffering of whole steps.  Two slots, each with its
+    own staged inputs (a StepIO), Decoder, pinned host outputs and step graph;
+    step i runs in slot i % 2.  The inputs of a step go up on one copy stream
+    while the previous step computes, and its outputs come back on another
+    while the next one computes.  Events order every reuse of a slot:
+      upload(i)   after compute(i - 2) has read the slot's inputs,
+      compute(i)  after upload(i) and after download(i - 2) has read the
+                  slot's outputs,
+      download(i) after compute(i).
+    `calls[s]` are slot s's pre-bound launches (bound to `compute`, reading
+    ios[s].dev and writing decs[s]'s buffers); `before(stream)`, if given,
+    enqueues work on the compute stream ahead of every step's graph.  Nothing
+    synchronises the host."""
+
+    def __init__(self, ios, decs, calls, compute: torch.cuda.Stream, before=None, nq: int | None = None):
+        assert len(ios) == len(decs) == len(calls) == 2
+        self.ios, self.decs, self.compute, self.before = ios, decs, compute, before
+        self.nq = decs[0].max_nq if nq is None else nq
+        self.up_stream = torch.cuda.Stream(device=compute.device)
+        self.down_stream = torch.cuda.Stream(device=compute.device)
+        self.hosts = [d.host_outputs() for d in decs]
+        self.graphs = [StepGraph(c, compute) for c in calls]
+        self._up = [torch.cuda.Event() for _ in range(2)]
+        self._done = [torch.cuda.Event() for _ in range(2)]
+        self._down = [torch.cuda.Event() for _ in range(2)]
+        self._used = [False, False]
+        self.d2h_bytes = 0
+
+    def step(self, i: int):
+        """Enqueue step i (inputs already in ios[i % 2].host)."""
+        s = i % 2
+        if self._used[s]:
+            self.up_stream.wait_event(self._done[s])
+        self.ios[s].upload(self.up_stream)
+        self._up[s].record(self.up_stream)
+        self.compute.wait_event(self._up[s])
+        if self._used[s]:
+            self.compute.wait_event(self._down[s])
+        if self.before is not None:
+            self.before(self.compute)
+        self.graphs[s].replay()
+        self._done[s].record(self.compute)
+        self.down_stream.wait_event(self._done[s])
+        self.d2h_bytes = self.decs[s].download(self.hosts[s], self.nq, self.down_stream)
+        self._down[s].record(self.down_stream)
+        self._used[s] = True
+
+    def uploaded(self, i: int) -> bool:
+        """Whether step i's inputs have left ios[i % 2].host (the slot's host
+        inputs may be refilled for step i + 2 only then)."""
+        return self._up[i % 2].query()
+
+    def wait_outputs(self, i: int):
+        """Block the host until step i's outputs are in host memory; return them
+        as (out, lse).  Step i + 2 reuses the slot's host outputs."""
+        self._down[i % 2].synchronize()
+        return self.outputs(i)
+
+    def outputs(self, i: int):
+        """Host (out, lse) of step i: valid once its download has completed."""
+        _, out, lse = self.hosts[i % 2]
+        return out, lse
+
+
 def splits_bound(k: int, chunk_units: int) -> int:
     """Most KV chunks one (query, KV head) pair's k+1 unit slots can touch."""
     return (k + 1 + chunk_units - 2) // chunk_units + 1
