@@ -444,7 +444,7 @@ def bind_append_kv(cache: PagedCache, k_new, v_new, kidx_new, seq_id, pos, dev_s
 
 
 # ----------------------------------------------------------------------------
-# a decode step: the four calls on preallocated buffers
+# a decode step: its calls on preallocated buffers
 
 
 class Decoder:

@@ -124,3 +124,15 @@ def test_binding_rejects_host_tensors():
     with pytest.raises(ValueError):
         qsa.qsa_combine(torch.zeros(1, 2, 4, 256), torch.zeros(1, 2, 4), torch.zeros(1, 4, 256, dtype=torch.bfloat16),
                         torch.zeros(1, 4))
+
+
+def test_fused_selection_rule():
+    """The Decoder's choice of the fused indexer + selection: enough clusters
+    to fill the SMs, all resident at once, and a decode-shaped call."""
+    import sparse_attention_decode_03_b200 as qsa
+    pays = qsa.fused_selection_pays
+    assert pays(32, 32, 148, 33)          # batch-32 decode: 256 CTAs, one wave
+    assert not pays(64, 64, 148, 33)      # two waves of clusters
+    assert not pays(8, 8, 148, 33)        # 64 CTAs leave most SMs idle
+    assert not pays(24, 2, 148, 33)       # 12 queries per sequence: prefill-shaped, the tensor-core indexer
+    assert not pays(32, 32, 148, 0)       # shared memory does not fit
