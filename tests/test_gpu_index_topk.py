@@ -141,3 +141,37 @@ def test_fused_full_size_matches_oracle_rows(name):
     for row in rows:
         r = R.expect_query(wl, row)
         assert np.array_equal(sel[row, :cnt[row]], r["sel"]), f"{name} row {row}"
+
+
+def test_fused_bad_page_flags_and_matches_two_calls():
+    """A block-table entry outside the page pool: both forms set BAD_PAGE,
+    score that page's 16 blocks -inf and select the same blocks."""
+    wl = C.shrink(C.get("long"), [6000, 3000], page_perm=True, k_top=64)
+    st0 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cache = H.build_cache(wl, dev_status=st0)
+    inp = H.step_inputs(wl)
+    qsa.qsa_append_kv(cache, inp["k_new"], inp["v_new"], inp["kidx_new"], inp["seq_id"], inp["pos"], st0)
+    torch.cuda.synchronize()
+    assert int(st0.item()) == 0
+    cache.block_table[0, 5] = 10 ** 7
+    ld = cache.max_pages_per_seq * 16
+    res = []
+    for fused in (False, True):
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        sc = torch.full((wl.nq, ld), 3.0, dtype=torch.float32, device="cuda")
+        sel = torch.zeros((wl.nq, 64), dtype=torch.int32, device="cuda")
+        cnt = torch.zeros((wl.nq,), dtype=torch.int32, device="cuda")
+        if fused:
+            qsa.qsa_index_topk(cache, inp["q_idx"], inp["w"], inp["q_seq"], inp["q_pos"], 64, sc, sel, cnt, st)
+        else:
+            qsa.qsa_index_scores(cache, inp["q_idx"], inp["w"], inp["q_seq"], inp["q_pos"], sc, st)
+            qsa.qsa_topk_blocks(sc, inp["q_pos"], 64, sel, cnt, st)
+        torch.cuda.synchronize()
+        res.append((int(st.item()), sc, sel, cnt))
+    (s0, sc0, se0, c0), (s1, sc1, se1, c1) = res
+    assert s0 & 1 and s1 & 1
+    nb = ((inp["q_pos"].long() + 1) // 4).tolist()
+    assert torch.all(torch.isneginf(sc1[0, 80:96]))
+    for r in range(wl.nq):
+        assert torch.equal(sc0[r, :nb[r]].view(torch.int32), sc1[r, :nb[r]].view(torch.int32)), f"scores row {r}"
+    assert torch.equal(se0, se1) and torch.equal(c0, c1)
