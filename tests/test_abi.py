@@ -124,6 +124,16 @@ def test_binding_rejects_host_tensors():
     with pytest.raises(ValueError):
         qsa.qsa_combine(torch.zeros(1, 2, 4, 256), torch.zeros(1, 2, 4), torch.zeros(1, 4, 256, dtype=torch.bfloat16),
                         torch.zeros(1, 4))
+    i32 = dict(dtype=torch.int32)
+    with pytest.raises(ValueError):  # checked before the cache is touched
+        qsa.qsa_index_topk(None, torch.zeros(2, 8, 128, dtype=torch.bfloat16), torch.zeros(2, 8),
+                           torch.zeros(2, **i32), torch.zeros(2, **i32), 16, torch.zeros(2, 64),
+                           torch.zeros(2, 16, **i32), torch.zeros(2, **i32))
+    with pytest.raises(ValueError):
+        qsa.qsa_sparse_attention(None, torch.zeros(2, 4, 256, dtype=torch.bfloat16), torch.zeros(2, **i32),
+                                 torch.zeros(2, **i32), torch.zeros(2, 16, **i32), torch.zeros(2, **i32), 16, 0.0625,
+                                 16, 4, torch.zeros(2, 4, 4, 256), torch.zeros(2, 4, 4), torch.zeros(2, **i32),
+                                 torch.zeros(2, 4, 256, dtype=torch.bfloat16), torch.zeros(2, 4))
 
 
 def test_fused_selection_rule():
