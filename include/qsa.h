@@ -183,7 +183,8 @@ QSA_API int qsa_topk_blocks(const float* scores, int64_t scores_ld, const int32_
 
 /*
  * qsa_index_topk -- qsa_index_scores followed by qsa_topk_blocks, in one
- * kernel: the same scores (bit for bit) and the same selections and counts.
+ * kernel ([DCP]: the indexer scores the micro-blocks and the best 512 are
+ * kept): the same scores (bit for bit) and the same selections and counts.
  * The score row of a query stays in on-chip shared memory, spread over a
  * cluster of 8 CTAs, while it is selected from, instead of being read back
  * from global memory; scores[q][j < nb_q] is still written.
@@ -269,7 +270,8 @@ QSA_API int qsa_sparse_decode(const qsa_cache_t* cache, const void* q, int32_t n
  * that pair's splits into out / lse with qsa_combine's arithmetic, so out and
  * lse equal those of the two calls bit for bit.
  *   pair_done int32 [nq][Hkv], all zero on entry; the call leaves it all zero
- *             (after a QSA_DEV_TIMEOUT status the caller must zero it again)
+ *             (after a QSA_DEV_TIMEOUT status the caller must zero it again);
+ *             calls sharing one pair_done must not overlap on the GPU
  *   out bf16 [nq][hq][256] (8-byte aligned); lse fp32 [nq][hq]
  * Other arguments, rules and errors: those of qsa_sparse_decode.
  */
