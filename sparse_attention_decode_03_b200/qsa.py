@@ -470,8 +470,11 @@ class Decoder:
             target_ctas = sms
         self.scores_ld = scores_ld or cache.max_pages_per_seq * BLOCKS_PER_PAGE
         if fused is None:
-            fused = (cache.kc_pages is not None and fused_selection_pays(
-                max_nq, cache.max_seqs, sms, index_topk_resident_queries(cache, self.scores_ld)))
+            try:  # a device without room for the clusters (or without clusters) keeps the two calls
+                resident = index_topk_resident_queries(cache, self.scores_ld) if cache.kc_pages is not None else 0
+            except QSAError:
+                resident = 0
+            fused = fused_selection_pays(max_nq, cache.max_seqs, sms, resident)
         self.fused = bool(fused)
         if chunk_units is None:
             chunk_units, self.max_splits = qsa_decode_plan(max_nq, cache.num_kv_heads, k, target_ctas)
