@@ -89,12 +89,20 @@ typedef enum {
  * One cache group ([DCP]: the selector and the main KV cache are kept in one
  * cache group so they cannot drift apart).  The main K/V and the compressed
  * indexer side cache are paged by the SAME physical page ids.
- *   kv_pages    [num_pages][num_kv_heads][16][2][4][256] elements of type
- *               kv_dtype, post-RoPE K and V: per page and KV head, its 16
- *               micro-blocks of 4 tokens, each holding the 4 K rows then the 4
- *               V rows, so one selected micro-block of one KV head is a single
- *               contiguous run (4 KiB in BF16, 2 KiB in FP8)
- *               (token t of a page: micro-block t / 4, row t % 4)
+ *   kv_pages    post-RoPE K and V of type kv_dtype: per page and KV head, its
+ *               16 micro-blocks of 4 tokens (token t of a page: micro-block
+ *               t / 4, row t % 4), each one contiguous run, so one selected
+ *               micro-block of one KV head is one copy:
+ *                 BF16: [num_pages][num_kv_heads][16] runs of 4 KiB, each
+ *                   [4 dim atoms][8 rows][64 elements]: atom a holds dims
+ *                   64a .. 64a+63 of rows 0-3 = K rows 0-3 and rows 4-7 =
+ *                   V rows 0-3 (128 B per row), and the 16-byte chunk c
+ *                   (elements 8c .. 8c+7) of row r sits at chunk position
+ *                   c XOR r of that row (the tensor cores' 128-byte swizzled
+ *                   operand layout, so a run is gathered into shared memory
+ *                   as it is);
+ *                 FP8: [num_pages][num_kv_heads][16][2][4][256] bytes: the 4 K
+ *                   rows then the 4 V rows (2 KiB per run).
  *   kc_pages    bf16 [num_pages][16][128]  kc of the 16 micro-blocks of a page
  *   kc_partial  fp32 [max_seqs][128]       running fp32 sum of each sequence's
  *                                           open (incomplete) micro-block
@@ -132,7 +140,7 @@ QSA_API const char* qsa_status_string(int status);
 
 /* ABI version of this header (bumped on any signature change). */
 QSA_API int qsa_abi_version(void);
-#define QSA_ABI_VERSION 6
+#define QSA_ABI_VERSION 7
 
 /*
  * qsa_append_kv -- write n new tokens into the cache group.
@@ -251,10 +259,10 @@ QSA_API int qsa_decode_plan(int32_t nq, int32_t hkv, int32_t k, int32_t target_c
  * chunk_units >= 1, max_splits >= the value qsa_decode_plan reports for
  * (k, chunk_units), scale > 0 (the pages keep the D256 scale 1/16).
  * The kernel gathers each selected micro-block (4 K rows + 4 V rows of one KV
- * head: one contiguous 4 KiB run) with 16-byte async copies into shared memory
- * and runs QK^T and PV on the tensor cores with fp32 accumulation; the
- * softmax weights P enter PV as a BF16 hi + lo pair (about 17 significant
- * bits), so short token sets keep full accuracy.
+ * head: one contiguous run) into shared memory as it is, with 16-byte async
+ * copies, and runs QK^T and PV on the tensor cores with fp32 accumulation;
+ * the softmax weights P enter PV as a BF16 hi + lo pair (about 17
+ * significant bits), so short token sets keep full accuracy.
  */
 QSA_API int qsa_sparse_decode(const qsa_cache_t* cache, const void* q, int32_t nq, int32_t hq, const int32_t* q_seq,
                       const int32_t* q_pos, const int32_t* sel, const int32_t* count, int32_t k, float scale,

@@ -109,20 +109,24 @@ __global__ void __launch_bounds__(kWarps * 32) append_scatter_kernel(AppendArgs 
   const int slot = p % kPage;
   const int hkv = a.c.num_kv_heads;
   for (int h = 0; a.c.kv_pages && h < hkv; ++h) {  // no main K/V in a selector-only group
-    // [page][h][micro-block][K rows | V rows][256] elements
-    const size_t blk = (((size_t)page * hkv + h) * kBlocksPerPage + slot / kRatio) * (2 * kRatio * kHeadDim);
-    const size_t dst = blk + (size_t)(slot % kRatio) * kHeadDim + lane * 8;
+    const size_t unit = ((size_t)page * hkv + h) * kBlocksPerPage + slot / kRatio;  // micro-block of one KV head
+    const int i = slot % kRatio;                                                     // its row
     const size_t src = ((size_t)tok * hkv + h) * kHeadDim + lane * 8;
     const uint4 kv8 = *reinterpret_cast<const uint4*>(a.k_new + src);
     const uint4 vv8 = *reinterpret_cast<const uint4*>(a.v_new + src);
+    uint8_t* kv = static_cast<uint8_t*>(a.c.kv_pages);
     if (a.c.kv_dtype == QSA_KV_FP8_E4M3) {
-      uint8_t* kv = static_cast<uint8_t*>(a.c.kv_pages);
+      // [unit][K rows | V rows][256] bytes
+      const size_t dst = unit * (2 * kRatio * kHeadDim) + (size_t)i * kHeadDim + lane * 8;
       *reinterpret_cast<uint2*>(kv + dst) = bf16x8_to_e4m3x8(kv8);
       *reinterpret_cast<uint2*>(kv + dst + kRatio * kHeadDim) = bf16x8_to_e4m3x8(vv8);
     } else {
-      __nv_bfloat16* kv = static_cast<__nv_bfloat16*>(a.c.kv_pages);
-      *reinterpret_cast<uint4*>(kv + dst) = kv8;
-      *reinterpret_cast<uint4*>(kv + dst + kRatio * kHeadDim) = vv8;
+      // [unit][4 dim atoms][8 rows: K 0-3, V 0-3][128 B]: the lane's 16 bytes are
+      // chunk lane % 8 of atom lane / 8, stored at chunk position (lane % 8) ^ row
+      const size_t base = unit * 4096 + (size_t)(lane >> 3) * 1024;
+      const int kr = i, vr = kRatio + i;
+      *reinterpret_cast<uint4*>(kv + base + kr * 128 + (((lane & 7) ^ kr) << 4)) = kv8;
+      *reinterpret_cast<uint4*>(kv + base + vr * 128 + (((lane & 7) ^ vr) << 4)) = vv8;
     }
   }
   if (a.c.kc_pages && (p & 3) == 3) {  // this token closes micro-block p / 4

@@ -263,18 +263,34 @@ __device__ __forceinline__ bool warp_aborted(volatile int* abort_flag) {
   return __shfl_sync(0xffffffffu, v, 0) != 0;
 }
 
+// Where a lookup warp publishes the unit descriptors of each 32-unit batch.
+struct LookupQueue {
+  uint64_t* d_off;       // [kDescSlots][kBatch] byte offset of the unit in the K/V pages (kNoCopy: none)
+  uint32_t* d_rows;      // [kDescSlots][kBatch] mask of the unit's valid rows
+  uint32_t bar_dfull;    // kDescSlots mbarriers: batch written
+  uint32_t bar_dempty;   // kDescSlots mbarriers: batch taken by every copy warp
+  volatile int* abort_flag;
+  uint32_t unit_bytes;
+};
+
 // Resolves kRound batches per round: the selection loads of all of them are
 // issued together, then the page-table loads, so a round costs two dependent
-// global-load latencies for 4 x 32 units.
-template <bool F8>
-__device__ void lookup_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_t x1) {
-  QSA_DECODE_LAYOUT;
+// global-load latencies for 4 x 32 units.  The CTA's first selection entries
+// are loaded before the per-query loads return (their address needs only the
+// chunk's geometry), so the first round costs one latency less.
+__device__ void lookup_run(const DecodeArgs& a, const LookupQueue& L, int64_t x0, int64_t x1) {
   const int lane = threadIdx.x & 31;
-  uint64_t* d_off = reinterpret_cast<uint64_t*>(smem + kOffDescOff);
-  uint32_t* d_rows = reinterpret_cast<uint32_t*>(smem + kOffDescRows);
-  const uint32_t bar_dfull = smem_u32(smem + kOffBar) + 2 * kStages * 8;
-  const uint32_t bar_dempty = bar_dfull + kDescSlots * 8;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
+  uint64_t* d_off = L.d_off;
+  uint32_t* d_rows = L.d_rows;
+  const uint32_t bar_dfull = L.bar_dfull, bar_dempty = L.bar_dempty;
+  volatile int* abort_flag = L.abort_flag;
+  const int64_t n_slots = (int64_t)a.K + 1;
+  const int64_t pair0 = x0 / n_slots;
+  const int q_first = (int)(pair0 / a.hkv);
+  const int u_first = (int)(x0 - pair0 * n_slots);
+  int j_first = 0;
+  if (u_first + lane < a.K) j_first = a.sel[(size_t)q_first * a.K + u_first + lane];
+  bool first_round = true;
   BatchIter it;
   bool have = iter_begin(a, it, x0, x1);
   int b = 0;
@@ -306,7 +322,9 @@ __device__ void lookup_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int6
       j[r] = 0;
       if (r < nr && lane < i_valid[r]) {
         if (lane < i_main[r]) {
-          j[r] = a.sel[(size_t)q[r] * a.K + sel_base[r] + lane];
+          j[r] = (first_round && r == 0 && q[r] == q_first && sel_base[r] == u_first)
+                     ? j_first
+                     : a.sel[(size_t)q[r] * a.K + sel_base[r] + lane];
           ok[r] = true;
         } else {
           j[r] = nb[r];
@@ -314,6 +332,7 @@ __device__ void lookup_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int6
         }
       }
     }
+    first_round = false;
 #pragma unroll
     for (int r = 0; r < kRound; ++r) {
       if (ok[r] && lane < i_main[r] && (j[r] < 0 || j[r] >= nb[r])) {
@@ -341,7 +360,7 @@ __device__ void lookup_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int6
           flag(a.st, QSA_DEV_BAD_PAGE);
         } else {
           off = (((uint64_t)phys[r] * a.hkv + g[r]) * kBlocksPerPage + (uint64_t)(j[r] % kBlocksPerPage)) *
-                kUnitBytes;  // bytes
+                L.unit_bytes;  // bytes
           rows = lane < i_main[r] ? 0xFu : (1u << t[r]) - 1u;
         }
       }
@@ -352,6 +371,19 @@ __device__ void lookup_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int6
     }
     b += nr;
   }
+}
+
+template <bool F8>
+__device__ void lookup_warp(const DecodeArgs& a, uint8_t* smem, int64_t x0, int64_t x1) {
+  QSA_DECODE_LAYOUT;
+  LookupQueue L;
+  L.d_off = reinterpret_cast<uint64_t*>(smem + kOffDescOff);
+  L.d_rows = reinterpret_cast<uint32_t*>(smem + kOffDescRows);
+  L.bar_dfull = smem_u32(smem + kOffBar) + 2 * kStages * 8;
+  L.bar_dempty = L.bar_dfull + kDescSlots * 8;
+  L.abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
+  L.unit_bytes = kUnitBytes;
+  lookup_run(a, L, x0, x1);
 }
 
 template <bool F8>
@@ -438,14 +470,19 @@ __device__ __forceinline__ bool consumer_wait(const DecodeArgs& a, uint32_t bar,
 }
 
 // Log-sum-exp merge of the nspl splits of pair (q, g) into out / lse, by the
-// 256 consumer threads of the CTA that wrote the pair's last split: thread t
-// owns dims 4 (t % 64) .. + 3 of rows t / 64, t / 64 + 4, ... of the group.
-// The arithmetic is that of qsa_combine (same order over the splits), so the
-// result is the same bit for bit.  Partials of other CTAs are read from L2.
-__device__ __forceinline__ void merge_pair(const DecodeArgs& a, int q, int g, int nspl, int tid) {
+// `nthreads` threads (a multiple of 32) of the CTA that wrote the pair's last
+// split: thread t owns dims 4 (t % 64) .. + 3 of every row of the group it
+// visits (rows t / 64, t / 64 + nthreads / 64, ... with 64 or more threads;
+// with 32, dims 4t .. + 3 and 128 + 4t .. + 3 of every row).  The arithmetic is
+// that of qsa_combine (same order over the splits), so the result is the same
+// bit for bit.  Partials of other CTAs are read from L2.
+__device__ __forceinline__ void merge_pair(const DecodeArgs& a, int q, int g, int nspl, int tid,
+                                           int nthreads = kConsumerThreads) {
   const int G = a.G;
-  const int c4 = tid & 63;
-  for (int r = tid >> 6; r < G; r += kConsumerThreads / 64) {
+  const int per = nthreads >= 64 ? nthreads / 64 : 1;  // rows visited at once
+  for (int idx = nthreads >= 64 ? tid >> 6 : 0; idx < G * (nthreads >= 64 ? 1 : 2); idx += per) {
+    const int r = nthreads >= 64 ? idx : idx >> 1;
+    const int c4 = nthreads >= 64 ? (tid & 63) : (tid & 31) + 32 * (idx & 1);
     const int h = g * G + r;
     const float* pl = a.part_lse + (size_t)q * a.max_splits * a.hq + h;
     const float* po = a.part_o + ((size_t)q * a.max_splits * a.hq + h) * kHeadDim + 4 * c4;
@@ -873,6 +910,492 @@ int launch_decode(const DecodeArgs& a, int64_t grid, void* stream) {
                           static_cast<cudaStream_t>(stream), a);
 }
 
+// ================================================================== BF16 form
+//
+// The BF16 cache stores each micro-block of one KV head as one 4 KiB run:
+// [4 dim atoms][8 rows: K 0-3, V 0-3][64 elements], the 16-byte chunk c of row
+// r at chunk position c ^ r (128-byte swizzle); the copy warps move each
+// selected run to its shared-memory slot as it is, with 16-byte cp.async
+// copies from every lane (bulk copies of whole runs, one per run, kept fewer
+// bytes in flight per SM on B200: about 29 GB/s per SM against 43 for the
+// 16-byte copies, whatever the ring depth).
+// The consumers are those of the mma.sync form, with fragment addresses
+// chosen for the swizzled rows so that every 16-byte fragment read of a warp is
+// bank-conflict free:
+//   * S n-tile j, column n is token (unit 2j + (n & 1), row (n >> 1) ^ (n & 1));
+//     for k-step pair i the lane reads chunk 8 (i >> 1) + 2 tq + (i & 1) of it
+//     (the contraction index is permuted identically in Q and K);
+//   * the PV B fragment's k index 2tq + (L & 1) + 8 (L >> 1) is then token
+//     (unit L, row tq ^ (L & 1)); lane gq reads dims chunk
+//     kappa(gq) = (gq >> 1) | ((gq & 1) << 2) of each 64-dim group, so output
+//     column n of an n-tile is dim 8 kappa(n) + the n-tile's offset.
+// Q fragments stay in registers for a whole segment.
+namespace sdb {
+
+constexpr int kUnitsPerTileB = 4;                       // 16 tokens
+constexpr int kStagesB = 8;
+constexpr int kUnitBytesB = 4096;
+constexpr int kStageBytesB = kUnitsPerTileB * kUnitBytesB;  // 16 KiB
+constexpr int kCopyWarp0B = kConsumerWarps;             // warps 8, 9
+constexpr int kLookupWarpB = kConsumerWarps + kCopyWarps;  // warp 10
+constexpr int kThreadsB = (kLookupWarpB + 1) * 32;
+constexpr int kOffComb = kStagesB * kStageBytesB;
+constexpr int kOffMLB = kOffComb + kCombBytes;
+constexpr int kOffXB = kOffMLB + kPairs * 16 * 2 * 4;
+constexpr int kOffDescOffB = kOffXB + kPairs * 2 * 2 * 32 * 8 * 4;
+constexpr int kOffDescRowsB = kOffDescOffB + kDescSlots * kBatch * 8;
+constexpr int kOffMetaB = kOffDescRowsB + kDescSlots * kBatch * 4;
+constexpr int kOffBarB = (kOffMetaB + kStagesB * 4 + 7) & ~7;
+constexpr int kNumBarsB = 2 * kStagesB + 2 * kDescSlots;
+constexpr int kOffAbortB = kOffBarB + kNumBarsB * 8;
+constexpr int kSmemUsedB = kOffAbortB + 16;
+constexpr int kSmemBytesB = kSmemUsedB + 128;           // slack to align the ring to 128 B
+static_assert(kSmemBytesB <= 232448, "shared memory budget");
+static_assert(kStagesB % kPairs == 0 && kStagesB % kCopyWarps == 0, "tile ownership must repeat with the stage ring");
+
+struct Ctx {
+  uint8_t* smem;   // 128-B aligned
+  uint32_t ring;   // its shared address
+  uint32_t bar;    // full[kStagesB], empty[kStagesB], dfull[kDescSlots], dempty[kDescSlots]
+  volatile int* abort_flag;
+};
+
+// ------------------------------------------------------------------ copy warps
+
+// Tile T (4 runs) belongs to copy warp T % 2; every lane copies 16 bytes of each
+// 512-byte eighth of each run and arrives on the stage's mbarrier when its copies
+// land (cp.async.mbarrier.arrive.noinc); lane 0 also publishes the row mask.
+__device__ void copy_run(const DecodeArgs& a, const Ctx& c, int64_t x0, int64_t x1, int cw) {
+  const int lane = threadIdx.x & 31;
+  const uint64_t* d_off = reinterpret_cast<const uint64_t*>(c.smem + kOffDescOffB);
+  const uint32_t* d_rows = reinterpret_cast<const uint32_t*>(c.smem + kOffDescRowsB);
+  uint32_t* meta = reinterpret_cast<uint32_t*>(c.smem + kOffMetaB);
+  const uint32_t bar_full = c.bar, bar_empty = c.bar + kStagesB * 8;
+  const uint32_t bar_dfull = c.bar + 2 * kStagesB * 8, bar_dempty = bar_dfull + kDescSlots * 8;
+  const uint64_t policy = l2_policy_evict_first();
+  const char* kv = reinterpret_cast<const char*>(a.kv_bytes);
+  int64_t T = 0;
+  BatchIter it;
+  bool have = iter_begin(a, it, x0, x1);
+  for (int b = 0; have; ++b, have = iter_next(a, it)) {
+    const int slot = b % kDescSlots;
+    if (!warp_wait(a, bar_dfull + slot * 8, (uint32_t)((b / kDescSlots) & 1), c.abort_flag)) break;
+    const uint64_t off = d_off[slot * kBatch + lane];
+    const uint32_t rows = d_rows[slot * kBatch + lane];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_dempty + slot * 8);  // both copy warps arrive
+    const int n_units = min(kBatch, it.s.n_valid - it.ub);
+    const int tiles = (n_units + kUnitsPerTileB - 1) / kUnitsPerTileB;
+    bool stop = false;
+    for (int tb = 0; tb < tiles; ++tb, ++T) {
+      if ((int)(T % kCopyWarps) != cw) continue;
+      const int stage = (int)(T % kStagesB);
+      if (T >= kStagesB && !warp_wait(a, bar_empty + stage * 8, (uint32_t)((T / kStagesB - 1) & 1), c.abort_flag)) {
+        stop = true;
+        break;
+      }
+      if (warp_aborted(c.abort_flag)) {
+        stop = true;
+        break;
+      }
+      const bool mine = (lane >> 2) == tb && lane < n_units;
+      const uint32_t rowmask = __reduce_or_sync(0xffffffffu, mine ? (rows << ((lane & 3) * 4)) : 0u);
+      const uint32_t dst = c.ring + (uint32_t)stage * kStageBytesB + lane * 16;
+#pragma unroll
+      for (int u = 0; u < kUnitsPerTileB; ++u) {
+        const uint64_t uoff = __shfl_sync(0xffffffffu, off, (tb * kUnitsPerTileB + u) & 31);
+        if (tb * kUnitsPerTileB + u < n_units && uoff != kNoCopy) {
+          const char* src = kv + uoff + lane * 16;
+#pragma unroll
+          for (int q8 = 0; q8 < kUnitBytesB / 512; ++q8) cp_async16(dst + u * kUnitBytesB + q8 * 512, src + q8 * 512, policy);
+        }
+      }
+      if (lane == 0) {
+        meta[stage] = rowmask;
+        mbar_arrive(bar_full + stage * 8);
+      }
+      cp_async_arrive_noinc(bar_full + stage * 8);
+    }
+    if (stop) break;
+  }
+  // Never leave the CTA with copies in flight.
+  cp_async_wait_all();
+  __syncwarp();
+}
+
+// ------------------------------------------------------------------ consumers
+
+__device__ void consumers(const DecodeArgs& a, const Ctx& c, int64_t x0, int64_t x1) {
+  const int tid = threadIdx.x;  // 0..255
+  const int warp = tid >> 5, lane = tid & 31;
+  const int cp = warp >> 1;     // consumer pair: owns tiles T with T % 4 == cp
+  const int half = warp & 1;    // output dims [128 * half, 128 * half + 128)
+  const int gq = lane >> 2, tq = lane & 3;
+  const uint32_t bar_full = c.bar, bar_empty = c.bar + kStagesB * 8;
+  const uint32_t* meta = reinterpret_cast<const uint32_t*>(c.smem + kOffMetaB);
+  float* comb = reinterpret_cast<float*>(c.smem + kOffComb);
+  float* ml = reinterpret_cast<float*>(c.smem + kOffMLB);
+  volatile int* abort_flag = c.abort_flag;
+  const int64_t n_slots = (int64_t)a.K + 1;
+  const int G = a.G;
+
+  // K fragment of S n-tile j: token (unit 2j + (gq & 1), row kr); byte offsets of its
+  // chunk 8 (i >> 1) + 2 tq + (i & 1) for the warp's k-step pairs i = 4 half + ii
+  const int kr = (gq >> 1) ^ (gq & 1);
+  uint32_t koff[4];
+#pragma unroll
+  for (int ii = 0; ii < 4; ++ii) {
+    const int i = 4 * half + ii;
+    const int ch = 8 * (i >> 1) + 2 * tq + (i & 1);
+    koff[ii] = (uint32_t)((gq & 1) * kUnitBytesB + (ch >> 3) * 1024 + kr * 128 + (((ch & 7) ^ kr) << 4));
+  }
+  // V loads L = 0..3: token (unit L, row tq ^ (L & 1)) = smem row 4 + that, chunk
+  // kappa(gq) of the 64-dim group 2 half + qh
+  const int kap = (gq >> 1) | ((gq & 1) << 2);
+  uint32_t voff[4];
+#pragma unroll
+  for (int L = 0; L < 4; ++L) {
+    const int vr = kRatio + (tq ^ (L & 1));
+    voff[L] = (uint32_t)(L * kUnitBytesB + (2 * half) * 1024 + vr * 128 + ((kap ^ vr) << 4));
+  }
+  // mask bits of the lane's S columns 2tq + e of n-tile j: token (unit 2j + e, row tq ^ e)
+  const int mb00 = 0 * 4 + tq, mb01 = 1 * 4 + (tq ^ 1), mb10 = 2 * 4 + tq, mb11 = 3 * 4 + (tq ^ 1);
+
+  int64_t T_base = 0;
+  for (int64_t pair = x0 / n_slots; pair <= (x1 - 1) / n_slots; ++pair) {
+    const Seg s = make_seg(a, pair, x0, x1, tid == 0);
+    const int n_tiles = (s.n_valid + kUnitsPerTileB - 1) / kUnitsPerTileB;
+    // ---- Q fragments of this KV group (rows >= G are zero), for the whole segment
+    uint4 qa[4], qc[4];
+    {
+      const __nv_bfloat16* qrow = a.q + ((size_t)s.q * a.hq + (size_t)s.g * G) * kHeadDim;
+      const bool ra = s.query_ok && gq < G, rc = s.query_ok && gq + 8 < G;
+#pragma unroll
+      for (int ii = 0; ii < 4; ++ii) {
+        const int i = 4 * half + ii;
+        const int ch = 8 * (i >> 1) + 2 * tq + (i & 1);
+        qa[ii] = ra ? ldg_nc(qrow + (size_t)gq * kHeadDim + ch * 8) : make_uint4(0, 0, 0, 0);
+        qc[ii] = rc ? ldg_nc(qrow + (size_t)(gq + 8) * kHeadDim + ch * 8) : make_uint4(0, 0, 0, 0);
+      }
+    }
+
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    float o[16][4];
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+
+    // tile T (counted over the whole chunk) belongs to pair T % 4
+    const int first_ti = (int)(((int64_t)cp - T_base % kPairs + kPairs) % kPairs);
+    for (int ti = first_ti; ti < n_tiles; ti += kPairs) {
+      const int64_t T = T_base + ti;
+      const int stage = (int)(T % kStagesB);
+      if (!*abort_flag) consumer_wait(a, bar_full + stage * 8, (uint32_t)((T / kStagesB) & 1), abort_flag);
+      __syncwarp();  // reconverge before the warp-wide mma.sync
+      const uint32_t mask = meta[stage];
+      const uint32_t kb = c.ring + (uint32_t)stage * kStageBytesB;
+
+      // ---- S = Q K^T over this warp's half of the dims; the pair swaps the partial sums
+      float sa[2][4], sb[2][4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sa[j][e] = sb[j][e] = 0.f;
+#pragma unroll
+      for (int ii = 0; ii < 4; ++ii) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          float(&acc)[4] = (ii & 1) ? sb[j] : sa[j];
+          const uint4 kk = lds128(kb + j * 2 * kUnitBytesB + koff[ii]);
+          mma_bf16_16816(acc, qa[ii].x, qc[ii].x, qa[ii].y, qc[ii].y, kk.x, kk.y);
+          mma_bf16_16816(acc, qa[ii].z, qc[ii].z, qa[ii].w, qc[ii].w, kk.z, kk.w);
+        }
+      }
+      {
+        float* xb = reinterpret_cast<float*>(c.smem + kOffXB) + ((cp * 2 + (int)((T / kPairs) & 1)) * 2) * 256;
+        float4* mine = reinterpret_cast<float4*>(xb + (half * 32 + lane) * 8);
+        const float4 p0 = make_float4(sa[0][0] + sb[0][0], sa[0][1] + sb[0][1], sa[0][2] + sb[0][2], sa[0][3] + sb[0][3]);
+        const float4 p1 = make_float4(sa[1][0] + sb[1][0], sa[1][1] + sb[1][1], sa[1][2] + sb[1][2], sa[1][3] + sb[1][3]);
+        mine[0] = p0;
+        mine[1] = p1;
+        named_bar_sync(2 + cp, 64);  // the pair's two warps
+        const float4* other = reinterpret_cast<const float4*>(xb + ((1 - half) * 32 + lane) * 8);
+        const float4 o0 = other[0], o1 = other[1];
+        sa[0][0] = p0.x + o0.x; sa[0][1] = p0.y + o0.y; sa[0][2] = p0.z + o0.z; sa[0][3] = p0.w + o0.w;
+        sa[1][0] = p1.x + o1.x; sa[1][1] = p1.y + o1.y; sa[1][2] = p1.z + o1.z; sa[1][3] = p1.w + o1.w;
+      }
+      // ---- mask, online softmax (base-2 logits)
+      float z[2][4];
+      float r0 = -INFINITY, r1 = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const bool v0 = (mask >> (j ? mb10 : mb00)) & 1u;  // column 2tq
+        const bool v1 = (mask >> (j ? mb11 : mb01)) & 1u;  // column 2tq + 1
+        z[j][0] = v0 ? sa[j][0] * a.scale_log2 : -INFINITY;
+        z[j][1] = v1 ? sa[j][1] * a.scale_log2 : -INFINITY;
+        z[j][2] = v0 ? sa[j][2] * a.scale_log2 : -INFINITY;
+        z[j][3] = v1 ? sa[j][3] * a.scale_log2 : -INFINITY;
+        r0 = fmaxf(r0, fmaxf(z[j][0], z[j][1]));
+        r1 = fmaxf(r1, fmaxf(z[j][2], z[j][3]));
+      }
+      r0 = fmaxf(r0, __shfl_xor_sync(0xffffffffu, r0, 1));
+      r1 = fmaxf(r1, __shfl_xor_sync(0xffffffffu, r1, 1));
+      r0 = fmaxf(r0, __shfl_xor_sync(0xffffffffu, r0, 2));
+      r1 = fmaxf(r1, __shfl_xor_sync(0xffffffffu, r1, 2));
+      const float mn0 = fmaxf(m0, r0), mn1 = fmaxf(m1, r1);
+      // a tile whose units were all rejected as bad data keeps every logit at -inf
+      const float sub0 = mn0 == -INFINITY ? 0.f : mn0, sub1 = mn1 == -INFINITY ? 0.f : mn1;
+      const float al0 = exp2f(m0 - sub0), al1 = exp2f(m1 - sub1);
+      m0 = mn0;
+      m1 = mn1;
+      float pr[2][4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        pr[j][0] = exp2f(z[j][0] - sub0);
+        pr[j][1] = exp2f(z[j][1] - sub0);
+        pr[j][2] = exp2f(z[j][2] - sub1);
+        pr[j][3] = exp2f(z[j][3] - sub1);
+      }
+      l0 = l0 * al0 + ((pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]));
+      l1 = l1 * al1 + ((pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]));
+      if (al0 != 1.f || al1 != 1.f) {
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) {
+          o[nt][0] *= al0;
+          o[nt][1] *= al0;
+          o[nt][2] *= al1;
+          o[nt][3] *= al1;
+        }
+      }
+      // P = hi + lo, both BF16, so the PV product keeps ~17 significant bits of
+      // every weight (BF16 alone, 8 bits, is too coarse for short token sets)
+      uint32_t pa[4], pl[4];
+      split_bf16(pr[0][0], pr[0][1], pa[0], pl[0]);
+      split_bf16(pr[0][2], pr[0][3], pa[1], pl[1]);
+      split_bf16(pr[1][0], pr[1][1], pa[2], pl[2]);
+      split_bf16(pr[1][2], pr[1][3], pa[3], pl[3]);
+
+      // ---- O += P V for this warp's 128 dims: 16 n-tiles, k = the tile's 16 tokens
+      // V load L reads token (unit L, row tq ^ (L & 1)); rows outside the selection
+      // may hold stale or never-written data and are zeroed
+      const bool full = mask == 0xffffu;
+      const bool ok0 = (mask >> (0 * 4 + tq)) & 1u, ok1 = (mask >> (1 * 4 + (tq ^ 1))) & 1u;
+      const bool ok2 = (mask >> (2 * 4 + tq)) & 1u, ok3 = (mask >> (3 * 4 + (tq ^ 1))) & 1u;
+#pragma unroll
+      for (int qh = 0; qh < 2; ++qh) {
+        uint4 x0v = lds128(kb + voff[0] + qh * 1024);
+        uint4 x1v = lds128(kb + voff[1] + qh * 1024);
+        uint4 x2v = lds128(kb + voff[2] + qh * 1024);
+        uint4 x3v = lds128(kb + voff[3] + qh * 1024);
+        if (!full) {
+          if (!ok0) x0v = make_uint4(0, 0, 0, 0);
+          if (!ok1) x1v = make_uint4(0, 0, 0, 0);
+          if (!ok2) x2v = make_uint4(0, 0, 0, 0);
+          if (!ok3) x3v = make_uint4(0, 0, 0, 0);
+        }
+        const uint32_t a0[4] = {x0v.x, x0v.y, x0v.z, x0v.w};
+        const uint32_t a1[4] = {x1v.x, x1v.y, x1v.z, x1v.w};
+        const uint32_t a2[4] = {x2v.x, x2v.y, x2v.z, x2v.w};
+        const uint32_t a3[4] = {x3v.x, x3v.y, x3v.z, x3v.w};
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const uint32_t lo01 = __byte_perm(a0[r], a1[r], 0x5410);
+          const uint32_t hi01 = __byte_perm(a0[r], a1[r], 0x7632);
+          const uint32_t lo23 = __byte_perm(a2[r], a3[r], 0x5410);
+          const uint32_t hi23 = __byte_perm(a2[r], a3[r], 0x7632);
+          mma_bf16_16816(o[qh * 8 + 2 * r], pa[0], pa[1], pa[2], pa[3], lo01, lo23);
+          mma_bf16_16816(o[qh * 8 + 2 * r + 1], pa[0], pa[1], pa[2], pa[3], hi01, hi23);
+          mma_bf16_16816(o[qh * 8 + 2 * r], pl[0], pl[1], pl[2], pl[3], lo01, lo23);
+          mma_bf16_16816(o[qh * 8 + 2 * r + 1], pl[0], pl[1], pl[2], pl[3], hi01, hi23);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_empty + stage * 8);  // both warps of the pair arrive
+    }
+    T_base += n_tiles;
+
+    // ---- merge the 4 pairs' (m, l, O) and write the split partial
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    if (half == 0 && tq == 0) {  // both warps of a pair hold the same m and l
+      ml[(cp * 16 + gq) * 2 + 0] = m0;
+      ml[(cp * 16 + gq) * 2 + 1] = l0;
+      ml[(cp * 16 + gq + 8) * 2 + 0] = m1;
+      ml[(cp * 16 + gq + 8) * 2 + 1] = l1;
+    }
+    named_bar_sync(kBarConsumers, kConsumerThreads);
+    // this pair's weight for rows gq / gq+8, and the merged lse of those rows
+    float fac[2], lse_row[2];
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int row = gq + 8 * hr;
+      const float mine = hr ? m1 : m0;
+      float M = -INFINITY;
+      for (int w = 0; w < kPairs; ++w) M = fmaxf(M, ml[(w * 16 + row) * 2]);
+      fac[hr] = 0.f;
+      lse_row[hr] = -INFINITY;
+      if (M != -INFINITY) {
+        float L = 0.f;
+        for (int w = 0; w < kPairs; ++w) {
+          const float mw = ml[(w * 16 + row) * 2];
+          if (mw != -INFINITY) L += ml[(w * 16 + row) * 2 + 1] * exp2f(mw - M);
+        }
+        fac[hr] = mine != -INFINITY ? exp2f(mine - M) / L : 0.f;
+        lse_row[hr] = (M + log2f(L)) * 0.69314718055994530942f;
+      }
+    }
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
+      o[nt][0] *= fac[0];
+      o[nt][1] *= fac[0];
+      o[nt][2] *= fac[1];
+      o[nt][3] *= fac[1];
+    }
+    // n-tile 8 qh + e, column 2tq + f holds dim 128 half + 64 qh + 8 kappa(2tq + f) + e,
+    // kappa(2tq) = tq and kappa(2tq + 1) = tq + 4
+    auto store_rows = [&](float* base, int row_stride) {
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int row = gq + 8 * hr;
+        if (row >= G) continue;
+        const int cc = 2 * hr;
+#pragma unroll
+        for (int qh = 0; qh < 2; ++qh) {
+#pragma unroll
+          for (int f = 0; f < 2; ++f) {
+            float4* d4 = reinterpret_cast<float4*>(base + (size_t)row * row_stride + 128 * half + 64 * qh + 32 * f + 8 * tq);
+            d4[0] = make_float4(o[qh * 8 + 0][cc + f], o[qh * 8 + 1][cc + f], o[qh * 8 + 2][cc + f], o[qh * 8 + 3][cc + f]);
+            d4[1] = make_float4(o[qh * 8 + 4][cc + f], o[qh * 8 + 5][cc + f], o[qh * 8 + 6][cc + f], o[qh * 8 + 7][cc + f]);
+          }
+        }
+      }
+    };
+    auto add_rows = [&](const float* base) {
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int row = gq + 8 * hr;
+        if (row >= G) continue;
+        const int cc = 2 * hr;
+#pragma unroll
+        for (int qh = 0; qh < 2; ++qh) {
+#pragma unroll
+          for (int f = 0; f < 2; ++f) {
+            const float4* s4 = reinterpret_cast<const float4*>(base + row * kCombRow + 128 * half + 64 * qh + 32 * f + 8 * tq);
+            const float4 x0 = s4[0], x1 = s4[1];
+            o[qh * 8 + 0][cc + f] += x0.x; o[qh * 8 + 1][cc + f] += x0.y;
+            o[qh * 8 + 2][cc + f] += x0.z; o[qh * 8 + 3][cc + f] += x0.w;
+            o[qh * 8 + 4][cc + f] += x1.x; o[qh * 8 + 5][cc + f] += x1.y;
+            o[qh * 8 + 6][cc + f] += x1.z; o[qh * 8 + 7][cc + f] += x1.w;
+          }
+        }
+      }
+    };
+    // merge step 1: pairs 2, 3 hand their O to pairs 0, 1; step 2: pair 1 to pair 0
+    if (cp >= 2) store_rows(comb + (cp - 2) * 16 * kCombRow, kCombRow);
+    named_bar_sync(kBarConsumers, kConsumerThreads);
+    if (cp < 2) add_rows(comb + cp * 16 * kCombRow);
+    named_bar_sync(kBarConsumers, kConsumerThreads);
+    if (cp == 1) store_rows(comb, kCombRow);
+    named_bar_sync(kBarConsumers, kConsumerThreads);
+    const size_t row0 = ((size_t)s.q * a.max_splits + s.split) * a.hq + (size_t)s.g * G;
+    if (cp == 0) {
+      add_rows(comb);
+      store_rows(a.part_o + row0 * kHeadDim, kHeadDim);
+      if (half == 0 && tq == 0) {
+        if (gq < G) a.part_lse[row0 + gq] = lse_row[0];
+        if (gq + 8 < G) a.part_lse[row0 + gq + 8] = lse_row[1];
+      }
+    }
+    if (s.last_of_pair) {  // slots this pair never reaches: empty splits
+      for (int sp = s.split + 1; sp < a.max_splits; ++sp) {
+        const size_t r0 = ((size_t)s.q * a.max_splits + sp) * a.hq + (size_t)s.g * G;
+        for (int idx = tid; idx < G * 64; idx += kConsumerThreads)
+          *reinterpret_cast<float4*>(a.part_o + (r0 + (idx >> 6)) * kHeadDim + (idx & 63) * 4) =
+              make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int row = tid; row < G; row += kConsumerThreads) a.part_lse[r0 + row] = -INFINITY;
+      }
+    }
+    if (a.pair_done) {
+      // The CTA that writes a pair's last split merges the pair: every writer
+      // fences its partial stores, one thread counts the split (device-scope
+      // atomic) and fences again before the merge reads the other splits.
+      __threadfence();
+      named_bar_sync(kBarConsumers, kConsumerThreads);
+      volatile int* last_flag = reinterpret_cast<volatile int*>(ml);  // ml is free until the next segment ends
+      const int64_t base = pair * n_slots;
+      const int nspl = (int)((base + n_slots - 1) / a.chunk - base / a.chunk) + 1;
+      if (tid == 0) {
+        const int done = atomicAdd(a.pair_done + pair, 1);
+        const bool last = done == nspl - 1;
+        if (last) a.pair_done[pair] = 0;  // every other split has counted: ready for the next call
+        __threadfence();
+        *last_flag = last ? 1 : 0;
+      }
+      named_bar_sync(kBarConsumers, kConsumerThreads);
+      const bool last = *last_flag != 0;
+      named_bar_sync(kBarConsumers, kConsumerThreads);  // the flag is read before ml is written again
+      if (last) merge_pair(a, s.q, s.g, nspl, tid);
+    } else {
+      named_bar_sync(kBarConsumers, kConsumerThreads);  // comb and ml are read before the next segment writes them
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreadsB, 1) sparse_decode_bf16_kernel(DecodeArgs a) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  pdl_launch_dependents();
+  Ctx c;
+  c.ring = (smem_u32(smem_raw) + 127u) & ~127u;
+  c.smem = smem_raw + (c.ring - smem_u32(smem_raw));
+  c.bar = c.ring + kOffBarB;
+  c.abort_flag = reinterpret_cast<volatile int*>(c.smem + kOffAbortB);
+  const int64_t x0 = (int64_t)blockIdx.x * a.chunk;
+  const int64_t x1 = min(x0 + a.chunk, a.total_slots);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStagesB; ++i) {
+      mbar_init(c.bar + i * 8, kFullArrivals);        // full: copy completions + row mask published
+      mbar_init(c.bar + (kStagesB + i) * 8, 2);       // empty: both warps of the owning pair
+    }
+    for (int i = 0; i < kDescSlots; ++i) {
+      mbar_init(c.bar + (2 * kStagesB + i) * 8, 1);               // descriptors written (lookup warp)
+      mbar_init(c.bar + (2 * kStagesB + kDescSlots + i) * 8, kCopyWarps);  // descriptors taken (copy warps)
+    }
+    *c.abort_flag = 0;
+    fence_mbar_init();
+  }
+  pdl_wait_previous();  // the selection and counts come from the previous kernel
+  __syncthreads();
+  if (x0 >= x1) return;
+  const int warp = threadIdx.x >> 5;
+  if (warp >= kCopyWarp0B && warp < kCopyWarp0B + kCopyWarps) {
+    copy_run(a, c, x0, x1, warp - kCopyWarp0B);
+  } else if (warp == kLookupWarpB) {
+    LookupQueue L;
+    L.d_off = reinterpret_cast<uint64_t*>(c.smem + kOffDescOffB);
+    L.d_rows = reinterpret_cast<uint32_t*>(c.smem + kOffDescRowsB);
+    L.bar_dfull = c.bar + 2 * kStagesB * 8;
+    L.bar_dempty = L.bar_dfull + kDescSlots * 8;
+    L.abort_flag = c.abort_flag;
+    L.unit_bytes = kUnitBytesB;
+    lookup_run(a, L, x0, x1);
+  } else {
+    consumers(a, c, x0, x1);
+  }
+}
+
+int launch(const DecodeArgs& a, int64_t grid, void* stream) {
+  cudaError_t e = cudaFuncSetAttribute(sparse_decode_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytesB);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QSA_ERR_CUDA;
+  }
+  return qsa_host::launch(sparse_decode_bf16_kernel, dim3((unsigned)grid), dim3(kThreadsB), kSmemBytesB,
+                          static_cast<cudaStream_t>(stream), a);
+}
+
+}  // namespace sdb
+
 }  // namespace
 
 int32_t qsa_splits_bound(int32_t k, int32_t chunk);
@@ -926,7 +1449,8 @@ int decode_call(const qsa_cache_t* cache, const void* q, int32_t nq, int32_t hq,
   a.st = dev_status;
   const int64_t grid = (a.total_slots + a.chunk - 1) / a.chunk;
   if (grid > 0x7fffffff) return QSA_ERR_UNSUPPORTED;
-  return c.kv_dtype == QSA_KV_FP8_E4M3 ? launch_decode<true>(a, grid, stream) : launch_decode<false>(a, grid, stream);
+  if (c.kv_dtype == QSA_KV_FP8_E4M3) return launch_decode<true>(a, grid, stream);
+  return sdb::launch(a, grid, stream);
 }
 
 }  // namespace

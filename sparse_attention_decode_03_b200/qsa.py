@@ -127,11 +127,14 @@ class PagedCache:
     """Device buffers of one cache group: main K/V pages and the compressed-indexer
     side cache, paged by the same page ids, plus the per-sequence open-block sum.
 
-    kv_pages is [page][Hkv][16 micro-blocks][2 (K, V)][4 rows][256]: one selected
-    micro-block of one KV head is a contiguous run, 4 KiB in BF16 (kv_dtype
-    KV_BF16) or 2 KiB in FP8 e4m3 (KV_FP8_E4M3).  with_kv=False leaves out the
-    main K/V (a selector-only group), with_kc=False the side cache (a K/V-only
-    group, e.g. a DCP rank's shard)."""
+    kv_pages holds, per page and KV head, 16 micro-blocks of 4 tokens, each one
+    contiguous run (one selected micro-block of one KV head is one copy):
+    BF16 (kv_dtype KV_BF16): [page][Hkv][16][4 dim atoms][8 rows][64], rows 0-3
+    the K rows and 4-7 the V rows, the 16-byte chunk c of row r at chunk
+    position c ^ r (the tensor cores' 128-byte swizzled operand layout);
+    FP8 e4m3 (KV_FP8_E4M3): [page][Hkv][16][2 (K, V)][4 rows][256].
+    with_kv=False leaves out the main K/V (a selector-only group),
+    with_kc=False the side cache (a K/V-only group, e.g. a DCP rank's shard)."""
 
     def __init__(self, num_pages: int, max_seqs: int, max_pages_per_seq: int, num_kv_heads: int,
                  block_table: torch.Tensor | None = None, device="cuda", kv_dtype: int = KV_BF16,
@@ -144,8 +147,9 @@ class PagedCache:
         self.kv_dtype = int(kv_dtype)
         if not (with_kv or with_kc):
             raise ValueError("a cache group needs the main K/V, the side cache, or both")
-        self.kv_pages = torch.empty((num_pages, num_kv_heads, BLOCKS_PER_PAGE, 2, RATIO, HEAD_DIM),
-                                    dtype=_KV_TORCH[self.kv_dtype], device=dev) if with_kv else None
+        shape = ((num_pages, num_kv_heads, BLOCKS_PER_PAGE, 4, 2 * RATIO, HEAD_DIM // 4) if self.kv_dtype == KV_BF16
+                 else (num_pages, num_kv_heads, BLOCKS_PER_PAGE, 2, RATIO, HEAD_DIM))
+        self.kv_pages = torch.empty(shape, dtype=_KV_TORCH[self.kv_dtype], device=dev) if with_kv else None
         self.kc_pages = torch.empty((num_pages, BLOCKS_PER_PAGE, IDX_DIM), dtype=torch.bfloat16,
                                     device=dev) if with_kc else None
         self.kc_partial = torch.zeros((max_seqs, IDX_DIM), dtype=torch.float32, device=dev) if with_kc else None
@@ -164,12 +168,24 @@ class PagedCache:
                                        self.max_pages_per_seq, self.num_kv_heads, self.kv_dtype)
         return self._struct
 
+    def _rows(self, kv: int) -> torch.Tensor:
+        if self.kv_dtype != KV_BF16:
+            return self.kv_pages[:, :, :, kv].reshape(self.num_pages, self.num_kv_heads, PAGE_TOKENS, HEAD_DIM)
+        # [page][Hkv][blk][atom][row][chunk position][8]: row r's chunk c sits at position c ^ r
+        x = self.kv_pages.view(self.num_pages, self.num_kv_heads, BLOCKS_PER_PAGE, 4, 2 * RATIO, 8, 8)
+        r = torch.arange(2 * RATIO, device=x.device)
+        pos = (torch.arange(8, device=x.device)[None, :] ^ r[:, None])      # [row][chunk] -> position
+        x = torch.gather(x, 5, pos[None, None, None, None, :, :, None].expand(x.shape))
+        x = x[:, :, :, :, kv * RATIO:(kv + 1) * RATIO]                       # [page][Hkv][blk][atom][4][8][8]
+        return x.permute(0, 1, 2, 4, 3, 5, 6).reshape(self.num_pages, self.num_kv_heads, PAGE_TOKENS, HEAD_DIM)
+
     def k_view(self) -> torch.Tensor:
-        """K as [page][Hkv][64][256] (a strided view, for inspection)."""
-        return self.kv_pages[:, :, :, 0].reshape(self.num_pages, self.num_kv_heads, PAGE_TOKENS, HEAD_DIM)
+        """K as [page][Hkv][64][256] (a copy in logical order, for inspection)."""
+        return self._rows(0)
 
     def v_view(self) -> torch.Tensor:
-        return self.kv_pages[:, :, :, 1].reshape(self.num_pages, self.num_kv_heads, PAGE_TOKENS, HEAD_DIM)
+        """V as [page][Hkv][64][256] (a copy in logical order, for inspection)."""
+        return self._rows(1)
 
     @property
     def capacity_tokens(self) -> int:
@@ -259,6 +275,22 @@ def fused_selection_pays(nq: int, max_seqs: int, sms: int, resident: int) -> boo
     call is decode-shaped (fewer than 8 queries per sequence on average;
     prefill calls take the tensor-core query-tiled indexer)."""
     return nq * 8 >= sms and nq <= resident and nq < 8 * max_seqs
+
+
+def fused_default(cache: PagedCache, scores_ld: int, nq: int, sms: int) -> bool:
+    """The Decoder's default selection form for a step of up to nq queries.  A
+    device that cannot place the fused kernel's clusters (the occupancy query
+    fails, or the clusters do not fit) keeps the two calls; an invalid cache or
+    scores_ld is the caller's error and raises QSAError."""
+    if cache.kc_pages is None:
+        return False
+    try:
+        resident = index_topk_resident_queries(cache, scores_ld)
+    except QSAError as e:
+        if e.status not in (QSA_ERR_UNSUPPORTED, QSA_ERR_CUDA):
+            raise
+        resident = 0
+    return fused_selection_pays(nq, cache.max_seqs, sms, resident)
 
 
 def qsa_decode_plan(nq: int, hkv: int, k: int, target_ctas: int) -> tuple[int, int]:
@@ -470,11 +502,7 @@ class Decoder:
             target_ctas = sms
         self.scores_ld = scores_ld or cache.max_pages_per_seq * BLOCKS_PER_PAGE
         if fused is None:
-            try:  # a device without room for the clusters (or without clusters) keeps the two calls
-                resident = index_topk_resident_queries(cache, self.scores_ld) if cache.kc_pages is not None else 0
-            except QSAError:
-                resident = 0
-            fused = fused_selection_pays(max_nq, cache.max_seqs, sms, resident)
+            fused = fused_default(cache, self.scores_ld, max_nq, sms)
         self.fused = bool(fused)
         if chunk_units is None:
             chunk_units, self.max_splits = qsa_decode_plan(max_nq, cache.num_kv_heads, k, target_ctas)

@@ -25,7 +25,7 @@ def test_library_exports_every_declared_symbol():
     lib = ctypes.CDLL(qsa.LIB_PATH)
     for n in header_functions():
         assert hasattr(lib, n), n
-    assert qsa.ABI_VERSION == 6
+    assert qsa.ABI_VERSION == 7
     assert qsa.status_string(0) == "QSA_OK" and qsa.status_string(-3) == "QSA_ERR_CUDA"
 
 
@@ -146,3 +146,56 @@ def test_fused_selection_rule():
     assert not pays(8, 8, 148, 33)        # 64 CTAs leave most SMs idle
     assert not pays(24, 2, 148, 33)       # 12 queries per sequence: prefill-shaped, the tensor-core indexer
     assert not pays(32, 32, 148, 0)       # shared memory does not fit
+
+
+def test_fused_default_falls_back_only_when_clusters_cannot_be_placed(monkeypatch):
+    """The Decoder's default keeps the two-call selection when the occupancy
+    query fails (QSA_ERR_CUDA) or is unsupported, and raises a caller error
+    (QSA_ERR_INVALID_ARG) instead of hiding it."""
+    import sparse_attention_decode_03_b200 as qsa
+    from sparse_attention_decode_03_b200 import qsa as Q
+
+    class FakeCache:
+        kc_pages = object()
+        max_seqs = 32
+
+    def failing(code):
+        def f(cache, scores_ld):
+            raise qsa.QSAError("qsa_index_topk_resident_queries", code)
+        return f
+
+    monkeypatch.setattr(Q, "index_topk_resident_queries", failing(Q.QSA_ERR_CUDA))
+    assert Q.fused_default(FakeCache(), 8192, 32, 148) is False
+    monkeypatch.setattr(Q, "index_topk_resident_queries", failing(Q.QSA_ERR_UNSUPPORTED))
+    assert Q.fused_default(FakeCache(), 8192, 32, 148) is False
+    monkeypatch.setattr(Q, "index_topk_resident_queries", failing(Q.QSA_ERR_INVALID_ARG))
+    with pytest.raises(qsa.QSAError):
+        Q.fused_default(FakeCache(), 8192, 32, 148)
+    monkeypatch.setattr(Q, "index_topk_resident_queries", lambda cache, ld: 33)
+    assert Q.fused_default(FakeCache(), 8192, 32, 148) is True
+
+
+def test_bf16_cache_views_follow_the_header_layout():
+    """PagedCache.k_view / v_view undo the BF16 cache's operand layout stated in
+    include/qsa.h: per micro-block [4 dim atoms][8 rows: K 0-3, V 0-3][64], the
+    16-byte chunk c of row r stored at chunk position c ^ r."""
+    import torch
+    from sparse_attention_decode_03_b200 import qsa as Q
+
+    class Cache(Q.PagedCache):
+        def __init__(self):  # host buffers only: no device needed
+            self.num_pages, self.num_kv_heads, self.kv_dtype = 2, 2, Q.KV_BF16
+            self.kv_pages = torch.zeros((2, 2, 16, 4, 8, 64), dtype=torch.int32)
+
+    c = Cache()
+    g = torch.Generator().manual_seed(3)
+    K = torch.randint(0, 1 << 30, (2, 2, 64, 256), dtype=torch.int32, generator=g)
+    V = torch.randint(0, 1 << 30, (2, 2, 64, 256), dtype=torch.int32, generator=g)
+    raw = c.kv_pages.view(2, 2, 16, 4, 8, 8, 8)
+    for t in range(64):
+        blk, i = t // 4, t % 4
+        for d in range(256):
+            atom, ch, e = d // 64, (d % 64) // 8, d % 8
+            raw[:, :, blk, atom, i, ch ^ i, e] = K[:, :, t, d]
+            raw[:, :, blk, atom, 4 + i, ch ^ (4 + i), e] = V[:, :, t, d]
+    assert torch.equal(c.k_view(), K) and torch.equal(c.v_view(), V)

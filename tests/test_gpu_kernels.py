@@ -236,9 +236,8 @@ def test_topk_rows_match_oracle_on_every_path(kind, n, k, pad, nrows):
     """Sampled-threshold path (random rows) and its fallback (sorted rows, heavy
     ties, crowded tails overflow a warp's candidate list), aligned and
     misaligned row strides, -inf scores, rows of 513 .. 100,000 blocks; with
-    few queries (1024-thread blocks) and many (300 rows: 256-thread blocks)."""
-    if nrows > 2 and n > 32768:
-        pytest.skip("the many-query form is covered up to 32,768 blocks per row")
+    few queries (1024-thread blocks) and many (300 rows, more than two per SM:
+    256-thread blocks), the long rows of a 256K-token context included."""
     gen = torch.Generator().manual_seed(n * 7 + k + pad)
     rows = [_topk_rows(kind, n, gen), _topk_rows("random", n, gen)]
     rows += [rows[i % 2] if i % 5 else _topk_rows(kind, n, gen) for i in range(2, nrows)]

@@ -41,6 +41,19 @@ def build_cache(wl: C.Workload, device="cuda", chunk_tokens: int = 32768, dev_st
     return cache
 
 
+def build_cache_from_host(wl: C.Workload, device="cuda", dev_status=None) -> qsa.PagedCache:
+    """The same cache group as build_cache, for small workloads: every row is
+    generated on the host and uploaded in one copy per tensor and sequence, so
+    the device runs only the library's append kernels (no generator kernels)."""
+    cache = new_cache(wl, device)
+    for b, L in enumerate(wl.lengths):
+        pos = torch.arange(0, L, dtype=torch.int64)
+        up = lambda t: t.to(device, non_blocking=False)
+        qsa.qsa_append_kv(cache, up(C.k_rows(wl, b, pos)), up(C.v_rows(wl, b, pos)), up(C.kidx_rows(wl, b, pos)),
+                          up(torch.full((L,), b, dtype=torch.int32)), up(pos.to(torch.int32)), dev_status)
+    return cache
+
+
 def step_tokens(wl: C.Workload, device="cuda") -> dict:
     """The tokens one step appends: positions lengths[b] .. lengths[b]+new-1 of
     every sequence, sequence-major."""
