@@ -157,7 +157,13 @@ QSA_API int qsa_abi_version(void);
  * A block left incomplete stores its running sum in kc_partial[seq].
  * Rules: the tokens of one sequence are contiguous in the arrays and at
  * consecutive increasing positions, and calls for a sequence arrive in
- * position order (violations set QSA_DEV_BAD_ORDER).  Two kernels are
+ * position order.  Detected (QSA_DEV_BAD_ORDER): a token whose predecessor
+ * in the arrays belongs to the same sequence at a position other than its
+ * own minus one.  NOT detected: a sequence whose tokens form several runs
+ * within one call (other sequences' tokens between them), and calls that
+ * skip or repeat positions across calls; every K/V row is still written, but
+ * that sequence's kc_pages rows and kc_partial are then undefined (other
+ * sequences are unaffected).  Two kernels are
  * enqueued.  n = 0 is a no-op.
  */
 QSA_API int qsa_append_kv(const qsa_cache_t* cache, const void* k_new, const void* v_new, const void* kidx_new,

@@ -127,12 +127,29 @@ class DCPRank:
         _q.qsa_combine_f32(po, plse, self.o_rank[:nq], self.lse_rank[:nq], stream)
         return self.o_rank[:nq], self.lse_rank[:nq]
 
-    def gather(self, group=None):
-        """All-gather every rank's (o, lse) buffers into o_all / lse_all,
-        rank-major (whole max_nq-row buffers: one collective each)."""
+    def gather(self, group=None, nq: int | None = None):
+        """All-gather every rank's (o, lse) into o_all / lse_all, rank-major.
+
+        On an NCCL group the whole max_nq-row device buffers go through one
+        all_gather_into_tensor each.  On a gloo group (host transport, e.g. ranks
+        sharing one GPU or a CPU-only test) the rank's first nq rows (default
+        max_nq) are copied to the host, all-gathered there and copied back into
+        o_all / lse_all; the device-to-host copy waits for the attention of the
+        current stream."""
         import torch.distributed as dist
-        dist.all_gather_into_tensor(self.o_all, self.o_rank, group=group)
-        dist.all_gather_into_tensor(self.lse_all, self.lse_rank, group=group)
+        if dist.get_backend(group) != "gloo":
+            dist.all_gather_into_tensor(self.o_all, self.o_rank, group=group)
+            dist.all_gather_into_tensor(self.lse_all, self.lse_rank, group=group)
+            return
+        n = self.max_nq if nq is None else int(nq)
+        o, lse = self.o_rank[:n].cpu(), self.lse_rank[:n].cpu()
+        o_parts = [torch.empty_like(o) for _ in range(self.sh.n)]
+        l_parts = [torch.empty_like(lse) for _ in range(self.sh.n)]
+        dist.all_gather(o_parts, o, group=group)
+        dist.all_gather(l_parts, lse, group=group)
+        for j in range(self.sh.n):
+            self.o_all[j, :n].copy_(o_parts[j], non_blocking=False)
+            self.lse_all[j, :n].copy_(l_parts[j], non_blocking=False)
 
     def merge(self, nq: int, stream=None):
         """Log-sum-exp merge over the ranks: (out bf16 [nq][hq][256], lse [nq][hq])."""

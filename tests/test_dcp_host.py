@@ -1,7 +1,8 @@
 """DCP host logic on the CPU: the shard rule of the binding against the
 oracle's, shard block tables, and the cross-rank exchange with two gloo ranks
 (each rank computes its share with the oracle, the shares are all-gathered
-rank-major and merged by log-sum-exp, which must give the unsharded result)."""
+rank-major -- by torch.distributed and by the library's DCPRank.gather -- and
+merged by log-sum-exp, which must give the unsharded result)."""
 import os
 import socket
 
@@ -85,6 +86,20 @@ def _rank_main(rank, world, port, interleave):
         dist.all_gather(l_all, l_r)
         o_all = torch.stack(o_all).numpy()           # rank-major [R][nq][Hq][256]
         l_all = torch.stack(l_all).numpy()
+        # the library's exchange (DCPRank.gather, gloo: staged through host memory) on the same shares
+        from types import SimpleNamespace
+        from sparse_attention_decode_03_b200.dcp import DCPRank, DCPShard
+        nq, max_nq = len(queries), len(queries) + 2
+        fake = SimpleNamespace(sh=DCPShard(world, rank, interleave), max_nq=max_nq,
+                               o_rank=torch.zeros((max_nq,) + tuple(o_r.shape[1:]), dtype=o_r.dtype),
+                               lse_rank=torch.zeros((max_nq,) + tuple(l_r.shape[1:]), dtype=l_r.dtype),
+                               o_all=torch.full((world, max_nq) + tuple(o_r.shape[1:]), 7.0, dtype=o_r.dtype),
+                               lse_all=torch.full((world, max_nq) + tuple(l_r.shape[1:]), 7.0, dtype=l_r.dtype))
+        fake.o_rank[:nq] = o_r
+        fake.lse_rank[:nq] = l_r
+        DCPRank.gather(fake, nq=nq)
+        assert np.array_equal(fake.o_all[:, :nq].numpy(), o_all) and np.array_equal(fake.lse_all[:, :nq].numpy(), l_all)
+        assert torch.all(fake.o_all[:, nq:] == 7.0)    # rows past nq are not touched
         for i, r in enumerate(refs):
             o, lse = O.combine(o_all[:, i], l_all[:, i])
             assert np.allclose(o, r["o"], rtol=1e-12, atol=1e-12), (rank, i)

@@ -117,6 +117,48 @@ def test_append_kv_bit_exact(name, lengths):
             assert torch.all(cache.kc_pages[last, nb % 16:].float() == 512.0)
 
 
+def test_append_order_rules():
+    """The stated order rules of qsa_append_kv: a token whose predecessor in the
+    arrays is the same sequence at a non-consecutive position sets
+    QSA_DEV_BAD_ORDER; a sequence split into two runs within one call is not
+    detected, but every K/V row is written and the other sequence's rows, kc and
+    open-block sum stay exact."""
+    wl = C.shrink(C.get("tiny"), [40, 40])
+    # detected: sequence 0 jumps from position 5 to 7 inside one run
+    cache = H.new_cache(wl)
+    st = _status()
+    pos = torch.tensor([4, 5, 7], dtype=torch.int32)
+    qsa.qsa_append_kv(cache, C.k_rows(wl, 0, pos).cuda(), C.v_rows(wl, 0, pos).cuda(), C.kidx_rows(wl, 0, pos).cuda(),
+                      torch.zeros(3, dtype=torch.int32, device="cuda"), pos.cuda(), st)
+    torch.cuda.synchronize()
+    assert "BAD_ORDER" in qsa.dev_status_names(int(st.item()))
+    # not detected: A 0..5, B 0..9, A 6..9 in one call
+    cache = H.new_cache(wl)
+    st = _status()
+    runs = [(0, 0, 6), (1, 0, 10), (0, 6, 10)]
+    parts = []
+    for b, p0, p1 in runs:
+        pos = torch.arange(p0, p1)
+        parts.append((C.k_rows(wl, b, pos), C.v_rows(wl, b, pos), C.kidx_rows(wl, b, pos),
+                      torch.full((p1 - p0,), b, dtype=torch.int32), pos.to(torch.int32)))
+    cat = [torch.cat([p[i] for p in parts]).cuda() for i in range(5)]
+    qsa.qsa_append_kv(cache, *cat, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    bt = cache.block_table.cpu()
+    for b in range(2):
+        pos = torch.arange(10)
+        pg, row = bt[b, pos // 64].long(), pos % 64
+        assert torch.equal(cache.k_view().cpu()[pg, :, row].view(torch.int16), C.k_rows(wl, b, pos).view(torch.int16))
+        assert torch.equal(cache.v_view().cpu()[pg, :, row].view(torch.int16), C.v_rows(wl, b, pos).view(torch.int16))
+    kid = C.kidx_rows(wl, 1, torch.arange(10)).float().numpy()
+    j = torch.arange(2)
+    kc_b = cache.kc_pages.cpu()[bt[1, j // 16].long(), j % 16].float().numpy()
+    assert np.array_equal(kc_b.view(np.uint32), O.compress_keys(kid).view(np.uint32))
+    assert np.array_equal(cache.kc_partial[1].cpu().numpy().view(np.uint32),
+                          O.open_block_partial(kid).view(np.uint32))
+
+
 def test_append_chunking_is_bitwise_invariant():
     """kc and the open-block partial do not depend on how the tokens are split
     into calls (all at once vs one token per call)."""
