@@ -501,8 +501,8 @@ def run_native(args, rank, ws, local):
     if not (torch.equal(out_h.view(torch.int16), last.out.cpu().view(torch.int16))
             and torch.equal(lse_h.view(torch.int32), last.lse.cpu().view(torch.int32))):
         raise RuntimeError("pipelined e2e: host outputs differ from the device's")
-    # append scatter + append partial + (scores + top-K, or the fused kernel) + (attention + combine, or merged)
-    launches_per_step = 2 + (1 if dec.fused else 2) + (1 if dec.merged else 2)
+    # append + (scores + top-K, or the fused kernel) + (attention + combine, or merged)
+    launches_per_step = 1 + (1 if dec.fused else 2) + (1 if dec.merged else 2)
 
     # ---- roofline of the dominant kernel
     count = dec.count[:wl.nq].cpu().numpy()
@@ -687,7 +687,7 @@ def run_dcp(args, rank, ws, local):
                      "alg_bytes_per_launch": dec_bytes, "peak_kind": f"{peak_kind} (hbm_gbs)",
                      "ms": round(dec_ms, 5)},
         "rank0_selected_blocks": int(cl.sum()), "all_selected_blocks": int(rk.count[:nq].sum()),
-        "gpu_launches": 10 * args.steps,  # 2 + 1 + 1 appends and localisation, scores, top-K, localisation, attention, 2 merges
+        "gpu_launches": 9 * args.steps,  # 2 appends, 2 localisations, scores, top-K, attention, 2 merges
         "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)

@@ -163,7 +163,7 @@ QSA_API int qsa_abi_version(void);
  * within one call (other sequences' tokens between them), and calls that
  * skip or repeat positions across calls; every K/V row is still written, but
  * that sequence's kc_pages rows and kc_partial are then undefined (other
- * sequences are unaffected).  Two kernels are
+ * sequences are unaffected).  One kernel is
  * enqueued.  n = 0 is a no-op.
  */
 QSA_API int qsa_append_kv(const qsa_cache_t* cache, const void* k_new, const void* v_new, const void* kidx_new,

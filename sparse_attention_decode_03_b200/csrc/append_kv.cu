@@ -9,13 +9,16 @@
 // Huawei's Ascend ...", section "Wat de pull request daadwerkelijk toevoegt"
 // (-1 padding marks slots that must not be used).
 //
-// Two kernels, one warp per token:
-//   scatter: writes K/V rows; the token at position 4j+3 closes block j and
-//            writes kc row j (partial of earlier calls + this call's tokens);
-//   partial: the last token of a sequence's run, if its block is still open,
-//            writes the running sum to kc_partial.
-// Splitting the partial write into a second launch orders it after every read
-// of the old partial in the first one.
+// One kernel, one warp per token.  Every warp writes its token's K/V rows; a
+// token at position 4j+3 whose whole block lies inside its run (the same
+// sequence at consecutive positions in this call) writes kc row j.  The warp
+// of a run's first token owns the run's open-block state: it finds the run's
+// last token (warp-wide probes of 32 tokens, strides growing by 32), completes
+// the run's first block when that block began in an earlier call (kc_partial
+// + this call's tokens: kc row, or the new partial if the run ends inside it),
+// and writes the running sum of the block left open at the run's end to
+// kc_partial.  Only that warp reads or writes kc_partial[seq], so one launch
+// orders every read of the old sum before its replacement.
 #include "qsa_common.cuh"
 
 namespace {
@@ -83,7 +86,35 @@ __device__ __forceinline__ float4 block_sum(const AppendArgs& a, int64_t tok, in
   return acc;
 }
 
-__global__ void __launch_bounds__(kWarps * 32) append_scatter_kernel(AppendArgs a) {
+// Is token t part of the run of sequence `seq` that starts at token `first`,
+// position p0 (same sequence, consecutive positions)?
+__device__ __forceinline__ bool in_run(const AppendArgs& a, int64_t t, int64_t first, int seq, int p0) {
+  return t < a.n && a.seq_id[t] == seq && (int64_t)a.pos[t] == (int64_t)p0 + (t - first);
+}
+
+// Index of the last token of the run that starts at token `first` (warp-uniform).
+// Runs are contiguous, so the probes that lie in the run form a prefix: grow the
+// stride by 32 while all 32 probes are in, then narrow the first miss down.
+__device__ __forceinline__ int64_t run_end(const AppendArgs& a, int64_t first, int seq, int p0, int lane) {
+  int64_t base = first, stride = 1;
+  for (;;) {
+    const unsigned m = __ballot_sync(0xffffffffu, in_run(a, base + stride * (lane + 1), first, seq, p0));
+    if (m != 0xffffffffu) {
+      base += stride * (__ffs(~m) - 1);
+      break;
+    }
+    base += stride * 32;
+    stride *= 32;
+  }
+  while (stride > 1) {  // the probe at base + 32 * stride is outside the run
+    stride /= 32;
+    const unsigned m = __ballot_sync(0xffffffffu, in_run(a, base + stride * (lane + 1), first, seq, p0));
+    base += stride * (__ffs(~m) - 1);
+  }
+  return base;
+}
+
+__global__ void __launch_bounds__(kWarps * 32) append_kernel(AppendArgs a) {
   pdl_launch_dependents();
   pdl_wait_previous();
   const int lane = threadIdx.x & 31;
@@ -100,7 +131,9 @@ __global__ void __launch_bounds__(kWarps * 32) append_scatter_kernel(AppendArgs 
     if (lane == 0) flag(a.st, QSA_DEV_BAD_POS);
     return;
   }
-  if (lane == 0 && tok > 0 && a.seq_id[tok - 1] == seq && a.pos[tok - 1] != p - 1) flag(a.st, QSA_DEV_BAD_ORDER);
+  const bool prev_same_seq = tok > 0 && a.seq_id[tok - 1] == seq;
+  const bool run_start = !(prev_same_seq && a.pos[tok - 1] == p - 1);
+  if (lane == 0 && prev_same_seq && a.pos[tok - 1] != p - 1) flag(a.st, QSA_DEV_BAD_ORDER);
   const int page = a.c.block_table[(int64_t)seq * a.c.max_pages_per_seq + p / kPage];
   if (page < 0 || page >= a.c.num_pages) {
     if (lane == 0) flag(a.st, QSA_DEV_BAD_PAGE);
@@ -129,35 +162,34 @@ __global__ void __launch_bounds__(kWarps * 32) append_scatter_kernel(AppendArgs 
       *reinterpret_cast<uint4*>(kv + base + vr * 128 + (((lane & 7) ^ vr) << 4)) = vv8;
     }
   }
-  if (a.c.kc_pages && (p & 3) == 3) {  // this token closes micro-block p / 4
-    const int m = run_before(a, tok, seq, p, 3);
-    const float4 acc = block_sum(a, tok, seq, m, m < 3, lane);
-    __nv_bfloat16* kc = static_cast<__nv_bfloat16*>(a.c.kc_pages) +
-                        ((size_t)page * kBlocksPerPage + slot / kRatio) * kIdxDim + lane * 4;
+  if (!a.c.kc_pages) return;
+  __nv_bfloat16* kc_page = static_cast<__nv_bfloat16*>(a.c.kc_pages) + (size_t)page * kBlocksPerPage * kIdxDim;
+  auto store_kc = [&](int blk_in_page, float4 acc) {
     uint2 out;
     out.x = pack_bf16(acc.x, acc.y);
     out.y = pack_bf16(acc.z, acc.w);
-    *reinterpret_cast<uint2*>(kc) = out;
+    *reinterpret_cast<uint2*>(kc_page + (size_t)blk_in_page * kIdxDim + lane * 4) = out;
+  };
+  // a block that lies wholly inside the run: its closing token writes kc
+  if ((p & 3) == 3 && run_before(a, tok, seq, p, 3) == 3) store_kc(slot / kRatio, block_sum(a, tok, seq, 3, false, lane));
+  if (!run_start) return;
+  // ---- the run's open-block state (this warp only)
+  const int64_t e = run_end(a, tok, seq, p, lane);
+  const int pe = p + (int)(e - tok);  // position of the run's last token
+  const int r0 = p & 3;
+  const int closer = p + (3 - r0);    // position closing the run's first block
+  if (r0 != 0) {  // the first block began in an earlier call: partial + this call's tokens
+    const int last = min(pe, closer);
+    const float4 acc = block_sum(a, tok + (last - p), seq, last - p, true, lane);
+    if (pe >= closer)
+      store_kc(slot / kRatio, acc);  // the block closes in this call (same page: blocks do not cross pages)
+    else
+      *reinterpret_cast<float4*>(a.c.kc_partial + (size_t)seq * kIdxDim + lane * 4) = acc;
   }
-}
-
-__global__ void __launch_bounds__(kWarps * 32) append_partial_kernel(AppendArgs a) {
-  pdl_launch_dependents();
-  pdl_wait_previous();  // every read of the old open-block sums (scatter kernel) is done
-  const int lane = threadIdx.x & 31;
-  const int64_t tok = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
-  if (tok >= a.n) return;
-  const int seq = a.seq_id[tok];
-  if (seq < 0 || seq >= a.c.max_seqs) return;
-  const int p = a.pos[tok];
-  if (p < 0 || (int64_t)p >= (int64_t)a.c.max_pages_per_seq * kPage) return;
-  const int r = p & 3;
-  if (r == 3) return;  // block closed by this token: nothing left open
-  const bool last = (tok == a.n - 1) || a.seq_id[tok + 1] != seq || a.pos[tok + 1] != p + 1;
-  if (!last) return;
-  const int m = run_before(a, tok, seq, p, r);
-  const float4 acc = block_sum(a, tok, seq, m, m < r, lane);
-  *reinterpret_cast<float4*>(a.c.kc_partial + (size_t)seq * kIdxDim + lane * 4) = acc;
+  if ((pe & 3) != 3 && (r0 == 0 || pe > closer)) {  // a block left open that began in this call
+    const float4 acc = block_sum(a, e, seq, pe & 3, false, lane);
+    *reinterpret_cast<float4*>(a.c.kc_partial + (size_t)seq * kIdxDim + lane * 4) = acc;
+  }
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -191,7 +223,5 @@ extern "C" int qsa_append_kv(const qsa_cache_t* cache, const void* k_new, const 
                dev_status};
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   const unsigned grid = (unsigned)((n + kWarps - 1) / kWarps);
-  int rc = qsa_host::launch(append_scatter_kernel, dim3(grid), dim3(kWarps * 32), 0, s, a);
-  if (rc != QSA_OK || !has_kc) return rc;
-  return qsa_host::launch(append_partial_kernel, dim3(grid), dim3(kWarps * 32), 0, s, a);
+  return qsa_host::launch(append_kernel, dim3(grid), dim3(kWarps * 32), 0, s, a);
 }

@@ -24,9 +24,8 @@ struct CombineArgs {
   float* lse;
 };
 
-// One CTA per (query, head).  Each thread recomputes the S split weights (S
-// lse values, broadcast from L1) and accumulates its 4 dims over the splits
-// with independent 16-byte loads.
+// One CTA per (query, head).  Each thread owns 4 dims; the split loads are
+// issued together (merge_row).
 template <bool F32Out>
 __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
   pdl_launch_dependents();
@@ -35,30 +34,11 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
   const int q = qh / a.hq, h = qh % a.hq;
   const int tid = threadIdx.x;
   const float* pl = a.part_lse + q * a.l_q + h;
-  float M = -INFINITY;
-  for (int s = 0; s < a.S; ++s) M = fmaxf(M, pl[s * a.l_s]);
-  float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
-  float lse_v = -INFINITY;
-  if (M != -INFINITY) {  // else every split is empty: zero output, lse = -inf
-    float L = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float* po = a.part_o + q * a.o_q + (int64_t)h * kHeadDim + 4 * tid;
-#pragma unroll 4
-    for (int s = 0; s < a.S; ++s) {
-      const float v = pl[s * a.l_s];
-      if (v == -INFINITY) continue;
-      const float e = expf(v - M);
-      const float4 x = *reinterpret_cast<const float4*>(po + s * a.o_s);
-      L += e;
-      acc.x += e * x.x;
-      acc.y += e * x.y;
-      acc.z += e * x.z;
-      acc.w += e * x.w;
-    }
-    const float inv = 1.f / L;
-    res = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-    lse_v = M + logf(L);
-  }
+  const float* po = a.part_o + q * a.o_q + (int64_t)h * kHeadDim + 4 * tid;
+  float lse_v;
+  const float4 res = merge_row(
+      a.S, [&](int s) { return pl[s * a.l_s]; },
+      [&](int s) { return *reinterpret_cast<const float4*>(po + s * a.o_s); }, lse_v);
   if constexpr (F32Out) {
     reinterpret_cast<float4*>(static_cast<float*>(a.out) + (size_t)qh * kHeadDim)[tid] = res;
   } else {

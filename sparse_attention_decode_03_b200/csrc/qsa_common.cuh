@@ -124,6 +124,64 @@ QSA_DEVINL void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
   lo = pack_bf16(a - ah, b - bh);
 }
 
+// ---------------------------------------------------------------- split merge
+// Log-sum-exp merge of split partials, in split order: with M = max lse,
+// L += e_s and acc += e_s * x_s for e_s = exp(lse_s - M), empty splits
+// (lse = -inf) skipped.  The separate combine and the attention kernel's
+// in-kernel merge both call this, so the two forms give identical bits.
+constexpr int kMergeBatch = 8;  // splits whose loads are issued together
+
+QSA_DEVINL void merge_splits(const float* v, const float4* x, int n, float M, float& L, float4& acc) {
+#pragma unroll
+  for (int s = 0; s < n; ++s) {
+    if (v[s] == -INFINITY) continue;
+    const float e = expf(v[s] - M);
+    L += e;
+    acc.x += e * x[s].x;
+    acc.y += e * x[s].y;
+    acc.z += e * x[s].z;
+    acc.w += e * x[s].w;
+  }
+}
+
+// One thread's 4 dims of one (query, head): the merged output (zero when every
+// split is empty) and the merged lse (-inf then).  Up to kMergeBatch splits,
+// every lse value and partial row is requested at once; more take a loop.
+// `lse_at(s)` / `row_at(s)` load split s.
+template <class LseAt, class RowAt>
+QSA_DEVINL float4 merge_row(int n, LseAt lse_at, RowAt row_at, float& lse_out) {
+  float M = -INFINITY, L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (n <= kMergeBatch) {
+    float v[kMergeBatch];
+    float4 x[kMergeBatch];
+#pragma unroll
+    for (int s = 0; s < kMergeBatch; ++s) v[s] = s < n ? lse_at(s) : -INFINITY;
+#pragma unroll
+    for (int s = 0; s < kMergeBatch; ++s)  // rows of empty splits are loaded but not used
+      x[s] = s < n ? row_at(s) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int s = 0; s < kMergeBatch; ++s) M = fmaxf(M, v[s]);
+    if (M != -INFINITY) merge_splits(v, x, kMergeBatch, M, L, acc);
+  } else {
+    for (int s = 0; s < n; ++s) M = fmaxf(M, lse_at(s));
+    if (M != -INFINITY) {
+      for (int s = 0; s < n; ++s) {
+        const float v = lse_at(s);
+        const float4 x = v == -INFINITY ? make_float4(0.f, 0.f, 0.f, 0.f) : row_at(s);
+        merge_splits(&v, &x, 1, M, L, acc);
+      }
+    }
+  }
+  if (M == -INFINITY) {
+    lse_out = -INFINITY;
+    return make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  const float inv = 1.f / L;
+  lse_out = M + logf(L);
+  return make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+}
+
 // ---------------------------------------------------------------- mbarrier + bulk copy
 
 QSA_DEVINL void mbar_init(uint32_t bar, uint32_t count) {

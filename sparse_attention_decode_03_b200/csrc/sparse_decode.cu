@@ -486,28 +486,10 @@ __device__ __forceinline__ void merge_pair(const DecodeArgs& a, int q, int g, in
     const int h = g * G + r;
     const float* pl = a.part_lse + (size_t)q * a.max_splits * a.hq + h;
     const float* po = a.part_o + ((size_t)q * a.max_splits * a.hq + h) * kHeadDim + 4 * c4;
-    float M = -INFINITY;
-    for (int sp = 0; sp < nspl; ++sp) M = fmaxf(M, __ldcg(pl + (size_t)sp * a.hq));
-    float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
-    float lse_v = -INFINITY;
-    if (M != -INFINITY) {  // else every split is empty: zero output, lse = -inf
-      float L = 0.f;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int sp = 0; sp < nspl; ++sp) {
-        const float v = __ldcg(pl + (size_t)sp * a.hq);
-        if (v == -INFINITY) continue;
-        const float e = expf(v - M);
-        const float4 x = __ldcg(reinterpret_cast<const float4*>(po + (size_t)sp * a.hq * kHeadDim));
-        L += e;
-        acc.x += e * x.x;
-        acc.y += e * x.y;
-        acc.z += e * x.z;
-        acc.w += e * x.w;
-      }
-      const float inv = 1.f / L;
-      res = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-      lse_v = M + logf(L);
-    }
+    float lse_v;
+    const float4 res = merge_row(
+        nspl, [&](int sp) { return __ldcg(pl + (size_t)sp * a.hq); },
+        [&](int sp) { return __ldcg(reinterpret_cast<const float4*>(po + (size_t)sp * a.hq * kHeadDim)); }, lse_v);
     uint2 o;
     o.x = pack_bf16(res.x, res.y);
     o.y = pack_bf16(res.z, res.w);
