@@ -32,6 +32,17 @@
  *    The library allocates nothing and never synchronises the host.
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream); calls only
  *    enqueue work on it.
+ *  - Kernels are launched with programmatic dependent launch: a kernel may
+ *    start before the preceding kernel of the stream has finished and waits
+ *    for it before it reads anything that kernel may write.  The indexer
+ *    calls (qsa_index_scores, qsa_index_topk) and qsa_topk_blocks read their
+ *    query inputs (q_seq, q_pos, q_idx, w) and the block table BEFORE that
+ *    wait.  They must therefore be complete by the time the preceding kernel
+ *    of the stream starts; when that kernel is qsa_append_kv, by the end of
+ *    the kernel before it (qsa_append_kv lets its dependents start only after
+ *    its own predecessor has finished).  Inputs written by host copies, or by
+ *    kernels that do not use programmatic dependent launch, earlier in the
+ *    stream always are.
  *  - Return value: QSA_OK, or a negative qsa_status for a host-detected error
  *    (nothing is enqueued then).
  *  - `dev_status` (may be NULL) is a device int32 the kernels OR error bits

@@ -115,8 +115,11 @@ __device__ __forceinline__ int64_t run_end(const AppendArgs& a, int64_t first, i
 }
 
 __global__ void __launch_bounds__(kWarps * 32) append_kernel(AppendArgs a) {
-  pdl_launch_dependents();
+  // The dependents may launch once this kernel's predecessor has finished:
+  // they read their query inputs before their own wait, and those may come
+  // from the kernel before this one.
   pdl_wait_previous();
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int64_t tok = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
   if (tok >= a.n) return;

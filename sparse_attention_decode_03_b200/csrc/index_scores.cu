@@ -43,32 +43,36 @@ struct ScoreArgs {
 
 __global__ void __launch_bounds__(kWarps * 32) index_scores_kernel(ScoreArgs a) {
   pdl_launch_dependents();
-  pdl_wait_previous();
   const int q = blockIdx.x / a.chunks_per_query;
   const int chunk = blockIdx.x % a.chunks_per_query;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
 
+  // The query's sequence, position, indexer query and page ids are inputs that
+  // no kernel of this library writes: they are loaded before waiting for the
+  // preceding kernel, so only the side-cache pages are read after the wait.
   const int seq = a.q_seq[q];
   const int p = a.q_pos[q];
-  if (seq < 0 || seq >= a.max_seqs || p < 0 || (int64_t)p >= (int64_t)a.mpps * kPage) {
-    if (chunk == 0 && threadIdx.x == 0) flag(a.st, (seq < 0 || seq >= a.max_seqs) ? QSA_DEV_BAD_SEQ : QSA_DEV_BAD_POS);
-    return;
-  }
-  int64_t nb = (p + 1) / kRatio;
-  if (nb > a.ld) {
-    if (chunk == 0 && threadIdx.x == 0) flag(a.st, QSA_DEV_SCORES_LD);
-    nb = a.ld;
-  }
+  const bool bad = seq < 0 || seq >= a.max_seqs || p < 0 || (int64_t)p >= (int64_t)a.mpps * kPage;
+  int64_t nb = bad ? 0 : (p + 1) / kRatio;
+  const bool ld_over = nb > a.ld;
+  if (ld_over) nb = a.ld;
   const int npg = (int)((nb + kBlocksPerPage - 1) / kBlocksPerPage);
   const int ppw = a.pages_per_warp;
   const int pg0 = chunk * (kWarps * ppw) + warp * ppw;
-  if (pg0 >= npg) return;
-
-  const IdxQuery Q = load_idx_query(a.q_idx, a.w, q);
-
+  IdxQuery Q{};
   int myphys = -1;
-  if (lane < ppw && pg0 + lane < npg) myphys = a.bt[(int64_t)seq * a.mpps + pg0 + lane];
+  if (!bad && pg0 < npg) {
+    Q = load_idx_query(a.q_idx, a.w, q);
+    if (lane < ppw && pg0 + lane < npg) myphys = a.bt[(int64_t)seq * a.mpps + pg0 + lane];
+  }
+  pdl_wait_previous();
+  if (bad) {
+    if (chunk == 0 && threadIdx.x == 0) flag(a.st, (seq < 0 || seq >= a.max_seqs) ? QSA_DEV_BAD_SEQ : QSA_DEV_BAD_POS);
+    return;
+  }
+  if (ld_over && chunk == 0 && threadIdx.x == 0) flag(a.st, QSA_DEV_SCORES_LD);
+  if (pg0 >= npg) return;
   float* srow = a.scores + (size_t)q * a.ld;
 
 #pragma unroll

@@ -106,10 +106,6 @@ __device__ __forceinline__ void st_cluster(void* p, uint32_t rank, uint32_t v) {
 }
 
 __global__ void __launch_bounds__(kFThreads, 2) index_topk_kernel(FusedArgs a) {
-  // The next kernel is allowed to launch only once every cluster has reached
-  // its selection (or left): launched earlier, its CTAs would take the shared
-  // memory this grid's later clusters need and push them into a second wave.
-  pdl_wait_previous();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   FSmem& S = *reinterpret_cast<FSmem*>(smem_raw);
   LocalLists& LL = *reinterpret_cast<LocalLists*>(smem_raw + kFOffLocal);
@@ -125,9 +121,31 @@ __global__ void __launch_bounds__(kFThreads, 2) index_topk_kernel(FusedArgs a) {
   const int K = a.K;
   int32_t* out = a.sel + (size_t)q * K;
 
+  // The query's sequence, position, indexer query and page ids are inputs that
+  // no kernel of this library writes: they are loaded before waiting for the
+  // preceding kernel, so only the side-cache pages are read after the wait.
   const int seq = a.q_seq[q];
   const int p = a.q_pos[q];
-  if (seq < 0 || seq >= a.max_seqs || p < 0 || (int64_t)p >= (int64_t)a.mpps * kPage) {
+  const bool bad = seq < 0 || seq >= a.max_seqs || p < 0 || (int64_t)p >= (int64_t)a.mpps * kPage;
+  int64_t nb = bad ? 0 : (p + 1) / kRatio;
+  const bool ld_over = nb > a.ld;
+  if (ld_over) nb = a.ld;
+  const int n = (int)nb;
+  const int npg = (n + kBlocksPerPage - 1) / kBlocksPerPage;
+  const int pps = (npg + kFC - 1) / kFC;  // pages per CTA (<= slice_pages: the host sizes the slice)
+  const int slice = pps * kBlocksPerPage;  // blocks per CTA
+  const int pg_lo = (int)rank * pps;
+  const int np_cta = max(0, min(npg, pg_lo + pps) - pg_lo);
+  const int b_lo = pg_lo * kBlocksPerPage;
+  const int m = max(0, min(n, b_lo + slice) - b_lo);  // blocks (keys) in this CTA's slice
+  const bool selecting = K > 0 && n > K;             // cluster-uniform
+  IdxQuery Q{};
+  if (!bad) {
+    for (int i = tid; i < np_cta; i += kFThreads) ids[i] = a.bt[(int64_t)seq * a.mpps + pg_lo + i];
+    if (np_cta > 0) Q = load_idx_query(a.q_idx, a.w, q);
+  }
+  pdl_wait_previous();
+  if (bad) {
     // the whole cluster leaves here, before any cluster barrier operation
     if (leader) {
       if (tid == 0) {
@@ -139,26 +157,11 @@ __global__ void __launch_bounds__(kFThreads, 2) index_topk_kernel(FusedArgs a) {
     return;
   }
   cluster_arrive_relaxed();  // this CTA is running (waited for before the first remote store)
-  int64_t nb = (p + 1) / kRatio;
-  if (nb > a.ld) {
-    if (leader && tid == 0) flag(a.st, QSA_DEV_SCORES_LD);
-    nb = a.ld;
-  }
-  const int n = (int)nb;
-  const int npg = (n + kBlocksPerPage - 1) / kBlocksPerPage;
-  const int pps = (npg + kFC - 1) / kFC;  // pages per CTA (<= slice_pages: the host sizes the slice)
-  const int slice = pps * kBlocksPerPage;  // blocks per CTA
-  const int pg_lo = (int)rank * pps;
-  const int np_cta = max(0, min(npg, pg_lo + pps) - pg_lo);
-  const int b_lo = pg_lo * kBlocksPerPage;
-  const int m = max(0, min(n, b_lo + slice) - b_lo);  // blocks (keys) in this CTA's slice
-  const bool selecting = K > 0 && n > K;             // cluster-uniform
+  if (ld_over && leader && tid == 0) flag(a.st, QSA_DEV_SCORES_LD);
 
   // ---------------- A. scores of this CTA's pages
-  for (int i = tid; i < np_cta; i += kFThreads) ids[i] = a.bt[(int64_t)seq * a.mpps + pg_lo + i];
-  __syncthreads();
+  __syncthreads();  // the page ids are in shared memory
   {
-    const IdxQuery Q = load_idx_query(a.q_idx, a.w, q);
     float* srow = a.scores + (size_t)q * a.ld;
     for (int pp = 2 * warp; pp < np_cta; pp += 2 * kFWarps) {  // warp-uniform
       uint4 ra[2][4], rb[2][4];
@@ -274,6 +277,9 @@ __global__ void __launch_bounds__(kFThreads, 2) index_topk_kernel(FusedArgs a) {
     if (tid == 0) st_cluster(&S.wcnt[rank], 0u, over ? (uint32_t)kFList + 1 : total);
   }
   cluster_barrier();  // 2: the leader holds every CTA's list; no shared memory is touched remotely after this
+  // The next kernel may launch only once every cluster has reached its
+  // selection (or left): launched earlier, its CTAs would take the shared
+  // memory this grid's later clusters need and push them into a second wave.
   pdl_launch_dependents();
   if (!leader) return;
 

@@ -72,12 +72,12 @@ __global__ void __launch_bounds__(kThreads, kThreads == kThreadsLarge ? 1 : 4) t
   constexpr int kWarps = kThreads / 32;
   constexpr int kSPer = kSample / kThreads;  // sample keys per thread
   pdl_launch_dependents();
-  pdl_wait_previous();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   TopkSmem<kWarps>& S = *reinterpret_cast<TopkSmem<kWarps>*>(smem_raw);
   const int q = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int p = a.q_pos[q];
+  const int p = a.q_pos[q];  // an input no kernel of this library writes: read before the wait
+  pdl_wait_previous();
   int64_t nb = p >= 0 ? (int64_t)(p + 1) / kRatio : 0;
   if (tid == 0 && p < 0) flag(a.st, QSA_DEV_BAD_POS);
   if (nb > a.ld) {

@@ -143,6 +143,9 @@ struct TopkSmem {
   uint32_t red[2 * kWarps];
   int bin;
   uint32_t above;
+  uint32_t nsmall;              // keys gathered from a small final bin
+  uint32_t skey[32], sidx[32];  // those keys and their block indices
+  uint32_t scut, sneed;         // the exact cut key, and how many keys equal to it are kept
 };
 
 // Add 1 to hist[bin] for every live lane.  Plain shared-memory atomics: the
@@ -289,6 +292,54 @@ __device__ uint32_t sample_threshold(const uint32_t (&ks)[kSPer], int ns, int n,
   return T0;
 }
 
+// The end of the exact select when the bin that holds the K-th key has at most
+// 32 keys: they are gathered (warp ballots, any order) and one warp ranks them
+// under (key desc, index asc), a total order, so the lane whose rank is
+// remaining - 1 holds the exact cut key whatever the gathering order.  On
+// return T is that key, M all ones and remaining the number of keys equal to
+// it that are kept (lowest index first).  Replaces the radix passes over the
+// lower bits.
+template <class Smem>
+__device__ void small_bin_cut(Smem& S, const uint32_t* ck, const uint32_t* ci, uint32_t mycnt, uint32_t mr,
+                              uint32_t& T, uint32_t& M, uint32_t& remaining) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  for (uint32_t j = lane; j < mr; j += 32) {
+    const bool in = j < mycnt && (ck[j] & M) == T;
+    const uint32_t b = __ballot_sync(0xffffffffu, in);
+    uint32_t base = 0;
+    if (lane == 0 && b) base = atomicAdd(&S.nsmall, (uint32_t)__popc(b));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    if (in) {
+      const uint32_t at = base + __popc(b & ((1u << lane) - 1u));
+      S.skey[at] = ck[j];
+      S.sidx[at] = ci[j];
+    }
+  }
+  __syncthreads();
+  if (tid < 32) {
+    const uint32_t n = S.nsmall;  // the bin's count, at most 32
+    const uint32_t key = lane < (int)n ? S.skey[lane] : 0u;
+    const uint32_t idx = lane < (int)n ? S.sidx[lane] : 0xffffffffu;
+    uint32_t rank = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const uint32_t kj = __shfl_sync(0xffffffffu, key, j), ij = __shfl_sync(0xffffffffu, idx, j);
+      rank += (j < (int)n && (kj > key || (kj == key && ij < idx))) ? 1u : 0u;
+    }
+    const uint32_t cut = __ballot_sync(0xffffffffu, lane < (int)n && rank == remaining - 1u);
+    const uint32_t Tk = __shfl_sync(0xffffffffu, key, __ffs(cut) - 1);
+    const uint32_t above = __popc(__ballot_sync(0xffffffffu, lane < (int)n && key > Tk));
+    if (lane == 0) {
+      S.scut = Tk;
+      S.sneed = remaining - above;
+    }
+  }
+  __syncthreads();
+  T = S.scut;
+  M = 0xffffffffu;
+  remaining = S.sneed;
+}
+
 // Steps 3 and 4: the exact top K among the candidates in the per-warp lists
 // S.ckey / S.cidx (S.wcnt[w] entries in list w; each list in block-index
 // order and the lists in index order by warp), written to out[0..K) in index
@@ -303,6 +354,7 @@ __device__ void select_from_lists(Smem& S, int K, int32_t* out) {
   const uint32_t* ck = S.ckey[warp];
   const uint32_t* ci = S.cidx[warp];
   const uint32_t mr = (mycnt + 31) & ~31u;
+  if (tid == 0) S.nsmall = 0;  // ordered before small_bin_cut by the barriers of block_minmax
 
   // ---- 3. exact select among the candidates
   uint32_t cmin = 0xffffffffu, cmax = 0u;
@@ -335,6 +387,10 @@ __device__ void select_from_lists(Smem& S, int K, int32_t* out) {
     M |= (uint32_t)(nbins - 1) << wlo;
     __syncthreads();
     if (remaining == in_bin) break;  // the whole bin is kept: its order does not matter
+    if (in_bin <= 32 && wlo > 0) {   // few keys left: rank them in one warp
+      small_bin_cut(S, ck, ci, mycnt, mr, T, M, remaining);
+      break;
+    }
     hb = wlo - 1;
   }
   const uint32_t need = remaining;  // keys equal to T (under M) to keep, lowest index first
