@@ -23,7 +23,7 @@
  * Fixed readings where the pages are silent: kc_j = sum of the 4 tokens'
  * indexer keys (fp32, token order, stored BF16 round-to-nearest-even);
  * s_j = sum_h w_h * ReLU(q_idx,h . kc_j) with 8 indexer heads of dim 128; ties
- * go to the lower block index; a query at position p sees nb = (p+1)/4
+ * (equal scores, -0 and +0 included) go to the lower block index; a query at position p sees nb = (p+1)/4
  * complete blocks and always attends its t = (p+1)%4 trailing tokens.
  *
  * Conventions for every call

@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(kFThreads, 2) index_topk_kernel(FusedArgs a) {
   if (selecting) {
     // the samples at positions i * n / ns that lie in this slice, to every CTA
     for (int i = tid; i < ns; i += kFThreads) {
-      const int pos = (int)((int64_t)i * n / ns);
+      const int pos = ns < kSample ? i : (int)((int64_t)i * n / kSample);  // ns is n or the constant kSample
       if (pos >= b_lo && pos < b_lo + m) {
         const uint32_t kv = keys[pos - b_lo];
 #pragma unroll

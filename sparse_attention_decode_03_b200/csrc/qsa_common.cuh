@@ -275,10 +275,22 @@ QSA_DEVINL void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// order-preserving map fp32 -> uint32 (larger float -> larger key)
+// order-preserving map fp32 -> uint32 (larger float -> larger key; equal
+// floats -> equal keys: -0 and +0 are the same score and share +0's key, so
+// they tie and the lower block index wins)
 QSA_DEVINL uint32_t float_key(float f) {
   uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// The float bound of a key threshold: float_key(x) >= T  <=>  x >= key_floor(T)
+// for every non-NaN x, when T lies between the keys of -inf and +inf.  For T in
+// the upper half (x >= +0) it is the float whose bits are T without the top
+// bit; below, the negative float whose key is T.  -0 >= +0 holds for floats,
+// as it does for the keys.
+QSA_DEVINL float key_floor(uint32_t T) {
+  return (T & 0x80000000u) ? __uint_as_float(T & 0x7fffffffu) : __uint_as_float(~T);
 }
 
 }  // namespace qsa

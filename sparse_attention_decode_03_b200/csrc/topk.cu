@@ -114,21 +114,26 @@ __global__ void __launch_bounds__(kThreads, kThreads == kThreadsLarge ? 1 : 4) t
 #pragma unroll
   for (int u = 0; u < kSPer; ++u) {
     const int i = u * kThreads + tid;
-    ks[u] = i < ns ? float_key(__ldg(s + (int64_t)i * n / ns)) : 0u;
+    // position i * n / ns; ns is either n (every key) or the constant kSample
+    const int64_t pos = ns < kSample ? (int64_t)i : (int64_t)i * n / kSample;
+    ks[u] = i < ns ? float_key(__ldg(s + pos)) : 0u;
   }
   const uint32_t T0 = sample_threshold<kThreads>(ks, ns, n, K, S);
 
-  // ---- 2. candidates: keys >= T0, per warp over its segment, in index order
+  // ---- 2. candidates: keys >= T0, per warp over its segment, in index order.
+  // The scores are compared as floats with T0's float bound; only the
+  // candidates' keys are computed.
+  const float thr = key_floor(T0);
   uint32_t cnt = 0;
   for (int c0 = w_lo; c0 < w_hi; c0 += kBatch * 128) {
     if (c0 != w_lo) load_batch(s, c0, w_hi, vec, v);
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int i0 = c0 + u * 128 + 4 * lane;
-      const uint32_t k[4] = {float_key(v[u].x), float_key(v[u].y), float_key(v[u].z), float_key(v[u].w)};
-      const bool f[4] = {i0 < w_hi && k[0] >= T0, i0 + 1 < w_hi && k[1] >= T0, i0 + 2 < w_hi && k[2] >= T0,
-                         i0 + 3 < w_hi && k[3] >= T0};
-      append4(S, warp, cnt, k, i0, f);
+      const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      const bool f[4] = {i0 < w_hi && x[0] >= thr, i0 + 1 < w_hi && x[1] >= thr, i0 + 2 < w_hi && x[2] >= thr,
+                         i0 + 3 < w_hi && x[3] >= thr};
+      append4_by(S, warp, cnt, [&](int c) { return float_key(x[c]); }, i0, f);
     }
   }
   if (lane == 0) S.wcnt[warp] = cnt > kCap ? kCap + 1 : cnt;

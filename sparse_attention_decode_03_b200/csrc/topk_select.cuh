@@ -224,30 +224,37 @@ __device__ int top_bin(const uint32_t* hist, int nbins, uint32_t remaining, Smem
   return b;
 }
 
-// Append lane's flagged keys (f0..f3 of idx0..idx0+3) to this warp's list, in index order.
-template <class Smem>
-__device__ __forceinline__ void append4(Smem& S, int warp, uint32_t& cnt, const uint32_t (&k)[4], int idx0,
-                                        const bool (&f)[4]) {
+// Append lane's flagged keys (f0..f3 of idx0..idx0+3) to this warp's list, in
+// index order.  A lane flags 0..4 keys, so the exclusive prefix of the counts
+// over the lanes comes from three ballots (one per bit of the count) and
+// popcounts, with no chain of shuffles.
+template <class Smem, class KeyAt>
+__device__ __forceinline__ void append4_by(Smem& S, int warp, uint32_t& cnt, KeyAt key_at, int idx0,
+                                           const bool (&f)[4]) {
   const int lane = threadIdx.x & 31;
   const uint32_t nc = (uint32_t)f[0] + f[1] + f[2] + f[3];
-  uint32_t inc = nc;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const uint32_t x = __shfl_up_sync(0xffffffffu, inc, d);
-    if (lane >= d) inc += x;
-  }
-  const uint32_t tot = __shfl_sync(0xffffffffu, inc, 31);
-  uint32_t pos = cnt + inc - nc;
+  const uint32_t b0 = __ballot_sync(0xffffffffu, nc & 1u);
+  const uint32_t b1 = __ballot_sync(0xffffffffu, nc & 2u);
+  const uint32_t b2 = __ballot_sync(0xffffffffu, nc & 4u);
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t pos = cnt + __popc(b0 & lt) + 2u * __popc(b1 & lt) + 4u * __popc(b2 & lt);
 #pragma unroll
   for (int c = 0; c < 4; ++c)
     if (f[c]) {
       if (pos < Smem::kList) {
-        S.ckey[warp][pos] = k[c];
+        S.ckey[warp][pos] = key_at(c);  // computed for flagged keys only
         S.cidx[warp][pos] = (uint32_t)(idx0 + c);
       }
       ++pos;
     }
-  cnt += tot;
+  cnt += __popc(b0) + 2u * __popc(b1) + 4u * __popc(b2);
+}
+
+// The same, for keys already held as keys.
+template <class Smem>
+__device__ __forceinline__ void append4(Smem& S, int warp, uint32_t& cnt, const uint32_t (&k)[4], int idx0,
+                                        const bool (&f)[4]) {
+  append4_by(S, warp, cnt, [&](int c) { return k[c]; }, idx0, f);
 }
 
 // Step 1: a threshold T0 such that about r >= K keys of the n-key row are

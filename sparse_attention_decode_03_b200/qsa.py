@@ -267,14 +267,17 @@ def index_topk_resident_queries(cache: PagedCache, scores_ld: int) -> int:
     return r
 
 
+FUSED_CLUSTER_CTAS = 8  # CTAs per query of qsa_index_topk (one cluster)
+
+
 def fused_selection_pays(nq: int, max_seqs: int, sms: int, resident: int) -> bool:
     """Whether a step of nq queries should run the fused indexer + selection:
-    its 8-CTA clusters fill the GPU (nq * 8 >= the SM count) and all fit at
-    once (nq <= resident: with a second wave the longest rows start late and
-    the two-call form, which spreads a row over many CTAs, is faster), and the
-    call is decode-shaped (fewer than 8 queries per sequence on average;
+    its clusters fill the GPU (nq * FUSED_CLUSTER_CTAS >= the SM count) and all
+    fit at once (nq <= resident: with a second wave the longest rows start late
+    and the two-call form, which spreads a row over many CTAs, is faster), and
+    the call is decode-shaped (fewer than 8 queries per sequence on average;
     prefill calls take the tensor-core query-tiled indexer)."""
-    return nq * 8 >= sms and nq <= resident and nq < 8 * max_seqs
+    return nq * FUSED_CLUSTER_CTAS >= sms and nq <= resident and nq < 8 * max_seqs
 
 
 def fused_default(cache: PagedCache, scores_ld: int, nq: int, sms: int) -> bool:

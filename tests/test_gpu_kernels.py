@@ -259,6 +259,8 @@ def _topk_rows(kind, n, gen):
         return -torch.arange(n, dtype=torch.float32)
     if kind == "ties":          # few distinct values: ties straddle the K-th key
         return torch.randint(0, 7, (n,), generator=gen).float()
+    if kind == "fine_ties":     # about 20 equal keys per value near the cut: a small last bin with ties
+        return torch.round(torch.randn(n, generator=gen) * 64) / 64
     if kind == "neg_inf":       # blocks whose page was rejected score -inf
         x = torch.randn(n, generator=gen)
         x[torch.rand(n, generator=gen) < 0.5] = float("-inf")
@@ -271,11 +273,12 @@ def _topk_rows(kind, n, gen):
 
 
 @pytest.mark.parametrize("nrows", [2, 300])
-@pytest.mark.parametrize("kind", ["random", "ascending", "descending", "ties", "neg_inf", "hot_tail"])
+@pytest.mark.parametrize("kind", ["random", "ascending", "descending", "ties", "fine_ties", "neg_inf", "hot_tail"])
 @pytest.mark.parametrize("n,k,pad", [(513, 512, 0), (1024, 512, 3), (1025, 1, 0), (4095, 2048, 1),
                                      (32768, 512, 0), (65536, 512, 5), (100000, 512, 0)])
 def test_topk_rows_match_oracle_on_every_path(kind, n, k, pad, nrows):
-    """Sampled-threshold path (random rows) and its fallback (sorted rows, heavy
+    """Sampled-threshold path (random rows; rows whose last radix bin is small
+    and holds ties straddling the K-th key) and its fallback (sorted rows, heavy
     ties, crowded tails overflow a warp's candidate list), aligned and
     misaligned row strides, -inf scores, rows of 513 .. 100,000 blocks; with
     few queries (1024-thread blocks) and many (300 rows, more than two per SM:

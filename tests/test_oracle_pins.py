@@ -195,6 +195,9 @@ def test_select_blocks_ties_and_edges():
     assert list(O.select_blocks(np.arange(10.0), 20)) == list(range(10))
     assert O.select_blocks(np.arange(10.0), 0).shape == (0,)
     assert list(O.select_blocks(np.array([1.0, 5.0, 5.0, 2.0, 5.0]), 2)) == [1, 2]
+    # -0 and +0 are the same score (IEEE equality): they tie and the lower index wins
+    assert list(O.select_blocks(np.array([-1.0, -0.0, 0.0]), 1)) == [1]
+    assert list(O.select_blocks(np.array([0.0, -1.0, -0.0, -0.0]), 2)) == [0, 2]
 
 
 # ---------------------------------------------------------------- attention
