@@ -354,24 +354,28 @@ __global__ void __launch_bounds__(kUThreads, 1) index_scores_umma_kernel(TiledAr
       int64_t B0, B1;
       pass_range(si, B0, B1);
       const int S = t_list[si];
+      // warp w copies chunks 4w .. 4w+3 of every row; lane l takes row 8k + (l & 7),
+      // chunk 4w + (l >> 3): one warp instruction writes 8 rows x 4 chunks, which the
+      // canonical layout puts in 4 lines of 8 distinct 16-byte bank groups (the
+      // minimum 4 wavefronts for 512 B), and reads 8 x 64 contiguous bytes.  A tile's
+      // page ids are loaded while the tile before it is copied, so no tile waits for
+      // a page-table round trip before its copies are issued.
+      constexpr int kPer = kTB * 16 / kUProdThreads;  // 16
+      const int c = 4 * (pt >> 5) + ((pt & 31) >> 3);
+      auto load_ids = [&](int64_t tb0, int (&ph)[kPer]) {
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+          const int64_t b = tb0 + 8 * k + (pt & 7);
+          ph[k] = b < B1 ? __ldg(a.bt + (int64_t)S * a.mpps + b / kBlocksPerPage) : -1;
+        }
+      };
+      int phys[kPer];
+      load_ids(B0, phys);
       for (int64_t b0 = B0; b0 < B1; b0 += kTB, ++j) {
         const int stage = j % kUStages;
         if (j >= kUStages && !uwait(bar_empty + stage * 8, (uint32_t)((j / kUStages - 1) & 1), abort_flag, a.st))
           break;
         const uint32_t tile = sb + kUOffA + stage * kUTileBytes;
-        // warp w copies chunks 4w .. 4w+3 of every row; lane l takes row 8k + (l & 7),
-        // chunk 4w + (l >> 3): one warp instruction writes 8 rows x 4 chunks, which the
-        // canonical layout puts in 4 lines of 8 distinct 16-byte bank groups (the
-        // minimum 4 wavefronts for 512 B), and reads 8 x 64 contiguous bytes.  The
-        // page ids are loaded first, all together (the copies are compiler barriers).
-        constexpr int kPer = kTB * 16 / kUProdThreads;  // 16
-        const int c = 4 * (pt >> 5) + ((pt & 31) >> 3);
-        int phys[kPer];
-#pragma unroll
-        for (int k = 0; k < kPer; ++k) {
-          const int64_t b = b0 + 8 * k + (pt & 7);
-          phys[k] = b < B1 ? __ldg(a.bt + (int64_t)S * a.mpps + b / kBlocksPerPage) : -1;
-        }
 #pragma unroll
         for (int k = 0; k < kPer; ++k) {
           const int r = 8 * k + (pt & 7);
@@ -385,6 +389,8 @@ __global__ void __launch_bounds__(kUThreads, 1) index_scores_umma_kernel(TiledAr
           }
         }
         cp_async_commit();
+        int next[kPer];  // the next tile's page ids, in flight during the waits below
+        load_ids(b0 + kTB, next);
         if (pend0 >= 0) {  // the copies of the tile issued two tiles ago have landed: publish it
           cp_async_wait_group<2>();
           fence_async_smem();
@@ -392,6 +398,8 @@ __global__ void __launch_bounds__(kUThreads, 1) index_scores_umma_kernel(TiledAr
         }
         pend0 = pend1;
         pend1 = j;
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) phys[k] = next[k];
       }
     }
     cp_async_wait_group<0>();
