@@ -129,6 +129,7 @@ struct TiledArgs {
   int32_t nq;
   float* scores;
   int64_t ld;
+  int32_t bulk;  // score rows 16-byte aligned (base and pitch): scores leave by bulk copies
   int32_t* st;
 };
 
@@ -147,11 +148,16 @@ __device__ __forceinline__ void cp_async_wait_group() {
 // q_idx[query][head] for the CTA's 32 queries, accumulated in tensor memory
 // (M = 128 blocks, N = 256, K = 128 dims in 8 steps of 16).  One TMEM lane per
 // block, so the w * ReLU head sum of a (query, block) score stays inside one
-// thread and the score stores are coalesced.
-//   warps 0-3  epilogue: tcgen05.ld of TMEM lanes 32w..32w+31, head sums, stores
-//   warp 4     TMEM allocation (512 columns: two accumulator buffers) and the
+// thread.
+//   warps 0-7  epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 (the lane
+//              quadrant a warp may access) and the columns of queries
+//              16 (w / 4) .. + 15, sums the heads, stages the scores in shared
+//              memory and stores each query's 32 consecutive scores with one
+//              128-byte bulk copy (cp.async.bulk, no multicast; element stores
+//              when the caller's score rows are not 16-byte aligned)
+//   warp 8     TMEM allocation (512 columns: two accumulator buffers) and the
 //              MMA issue (one elected thread), tcgen05.commit to mbarriers
-//   warps 5-8  producers: 16-byte cp.async of q_idx (once) and of every kc
+//   warps 9-12 producers: 16-byte cp.async of q_idx (once) and of every kc
 //              tile into the canonical K-major, no-swizzle operand layout
 //              (8-row x 16-byte core matrices; the two 8-element halves of a
 //              16-element K step 128 B apart, 8-row groups 256 B apart), then
@@ -163,8 +169,9 @@ __device__ __forceinline__ void cp_async_wait_group() {
 
 constexpr int kUStages = 4;
 constexpr int kUTileBytes = kTB * kIdxDim * 2;                 // 32 KiB: one operand of 128 rows
-constexpr int kUEpiWarps = 4, kUMmaWarp = 4, kUProdWarp0 = 5, kUProdWarps = 4;
-constexpr int kUThreads = (kUProdWarp0 + kUProdWarps) * 32;    // 288
+constexpr int kUEpiWarps = 8, kUMmaWarp = 8, kUProdWarp0 = 9, kUProdWarps = 4;
+constexpr int kUThreads = (kUProdWarp0 + kUProdWarps) * 32;    // 416
+constexpr int kUEpiQ = kTQ * 4 / kUEpiWarps;                    // queries per epilogue warp: 16
 constexpr int kUProdThreads = kUProdWarps * 32;
 constexpr int kUN = kTQ * kIdxHeads;                           // 256: MMA N = the CTA's queries x heads
 constexpr int kUBBytes = kUN * kIdxDim * 2;                    // 64 KiB: the q_idx operand
@@ -176,7 +183,9 @@ constexpr int kUOffW = kUOffA + kUStages * kUTileBytes;        // [32][8] weight
 constexpr int kUOffMeta = kUOffW + kTQ * kIdxHeads * 4;        // t_seq[32], t_nb[32], t_list[32], count, tmem, abort
 constexpr int kUOffBar = (kUOffMeta + (3 * kTQ + 4) * 4 + 7) & ~7;
 constexpr int kUNumBars = 2 * kUStages + 2 * kUAcc + 2;        // full/empty per stage, acc full/empty, b_full, done
-constexpr int kUSmem = kUOffBar + kUNumBars * 8;
+constexpr int kUStageFloats = kUEpiQ * 32;                     // one epilogue warp's 32 rows x 16 queries
+constexpr int kUOffStage = (kUOffBar + kUNumBars * 8 + 127) & ~127;  // 2 x 4 warps score staging buffers
+constexpr int kUSmem = kUOffStage + 2 * kUEpiWarps * kUStageFloats * 4;
 constexpr uint32_t kUIdesc = (1u << 4)                       // D: fp32
                            | (1u << 7) | (1u << 10)          // A, B: bf16
                            | ((uint32_t)(kUN >> 3) << 17)    // N = 256
@@ -219,7 +228,21 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// bulk copy shared -> global (16-byte aligned addresses, size a multiple of 16), tracked per thread in groups
+__device__ __forceinline__ void bulk_s2g(void* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// all but this thread's most recent group have finished reading their shared-memory source
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+// every group of this thread has completed its writes
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+__device__ __forceinline__ void reg_fence16(uint32_t (&r)[16]) {
+  asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+               "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]));
+}
 // bounded mbarrier wait shared by all roles; false once the CTA aborted
 __device__ __forceinline__ bool uwait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* st) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -437,8 +460,10 @@ __global__ void __launch_bounds__(kUThreads, 1) index_scores_umma_kernel(TiledAr
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue: row = block b0 + 32 * warp + lane
-    const int row = 32 * warp + lane;
+    // ---------------- epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 (rows) and the
+    // columns of queries 16 (w / 4) .. + 15
+    const int qd = warp & 3, qh = warp >> 2;
+    const int row = 32 * qd + lane;
     int j = 0;
     for (int si = 0; si < nseq; ++si) {
       int64_t B0, B1;
@@ -451,37 +476,68 @@ __global__ void __launch_bounds__(kUThreads, 1) index_scores_umma_kernel(TiledAr
         const int phys = b < B1 ? a.bt[(int64_t)S * a.mpps + b / kBlocksPerPage] : 0;
         if (!uwait(bar_accf + acc * 8, (uint32_t)((j / kUAcc) & 1), abort_flag, a.st)) goto epi_done;
         tc_fence_after();
-        float sc[kTQ];
-        const uint32_t taddr = tmem + acc * kUN + ((uint32_t)(32 * warp) << 16);
+        float sc[kUEpiQ];
+        const uint32_t taddr = tmem + acc * kUN + ((uint32_t)(32 * qd) << 16) + (uint32_t)(qh * kUEpiQ * kIdxHeads);
 #pragma unroll
-        for (int h8 = 0; h8 < kTQ / 8; ++h8) {  // 4 loads of two queries (16 columns) each, then one wait
+        for (int h8 = 0; h8 < kUEpiQ / 8; ++h8) {  // 4 loads of two queries (16 columns) each, then one wait
           uint32_t r[4][16];
 #pragma unroll
           for (int u = 0; u < 4; ++u) tmem_ld16(taddr + (h8 * 4 + u) * 16, r[u]);
           tmem_wait_ld();
 #pragma unroll
+          for (int u = 0; u < 4; ++u) reg_fence16(r[u]);
+#pragma unroll
           for (int u = 0; u < 4; ++u)
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
               const int ql = 2 * (h8 * 4 + u) + k;
+              const int qg = qh * kUEpiQ + ql;
+              const float4 wa = *reinterpret_cast<const float4*>(t_w + qg * kIdxHeads);
+              const float4 wb = *reinterpret_cast<const float4*>(t_w + qg * kIdxHeads + 4);
+              const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
               float s = 0.f;
 #pragma unroll
-              for (int hd = 0; hd < kIdxHeads; ++hd)
-                s += t_w[ql * kIdxHeads + hd] * relu(__uint_as_float(r[u][8 * k + hd]));
+              for (int hd = 0; hd < kIdxHeads; ++hd) s += wv[hd] * relu(__uint_as_float(r[u][8 * k + hd]));
               sc[ql] = s;
             }
         }
         tc_fence_before();
         mbar_arrive(bar_acce + acc * 8);  // this thread is done reading the accumulator
         const bool bad = b < B1 && (phys < 0 || phys >= a.num_pages);
+        if (a.bulk) {
+          float* stg = reinterpret_cast<float*>(smem + kUOffStage) + ((j & 1) * kUEpiWarps + warp) * kUStageFloats;
+          bulk_wait_read1();
+          __syncwarp();
 #pragma unroll
-        for (int ql = 0; ql < kTQ; ++ql) {
-          if (t_seq[ql] == S && b < t_nb[ql])
-            a.scores[(size_t)(q0 + ql) * a.ld + b] = bad ? -INFINITY : sc[ql];
+          for (int ql = 0; ql < kUEpiQ; ++ql) stg[ql * 32 + lane] = bad ? -INFINITY : sc[ql];
+          fence_async_smem();
+          __syncwarp();
+          const int64_t bw = b0 + 32 * qd;
+          if (lane < kUEpiQ) {
+            const int qg = qh * kUEpiQ + lane;
+            const int nbq = t_nb[qg];
+            if (t_seq[qg] == S && bw < nbq) {
+              float* dst = a.scores + (size_t)(q0 + qg) * a.ld + bw;
+              if (bw + 32 <= nbq) {
+                bulk_s2g(dst, smem_u32(stg + lane * 32), 128u);
+              } else {
+                for (int i = 0; i < nbq - bw; ++i) dst[i] = stg[lane * 32 + i];
+              }
+            }
+          }
+          bulk_commit();
+        } else {
+#pragma unroll
+          for (int ql = 0; ql < kUEpiQ; ++ql) {
+            const int qg = qh * kUEpiQ + ql;
+            if (t_seq[qg] == S && b < t_nb[qg])
+              a.scores[(size_t)(q0 + qg) * a.ld + b] = bad ? -INFINITY : sc[ql];
+          }
         }
       }
     }
   epi_done:;
+    bulk_wait_all();  // the scores are written before the CTA ends
   }
   tc_fence_before();
   __syncthreads();
@@ -531,6 +587,7 @@ extern "C" int qsa_index_scores(const qsa_cache_t* cache, const void* q_idx, con
     t.nq = nq;
     t.scores = scores;
     t.ld = scores_ld;
+    t.bulk = (reinterpret_cast<uintptr_t>(scores) & 15u) == 0 && (scores_ld & 3) == 0;
     t.st = dev_status;
     int64_t max_blocks = (int64_t)cache->max_pages_per_seq * kBlocksPerPage;
     if (scores_ld < max_blocks) max_blocks = scores_ld;

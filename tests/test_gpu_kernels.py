@@ -234,6 +234,33 @@ def test_query_tiled_index_scores_bit_exact(lengths, new, k):
         assert np.array_equal(sel[row, :cnt[row]], sel_ref), f"selection row {row}"
 
 
+def test_query_tiled_scores_any_row_pitch():
+    """The query-tiled indexer stores aligned score rows with bulk copies and
+    falls back to element stores when a row's start is not 16-byte aligned (an
+    odd pitch, or an offset base).  All three give the same scores, and no
+    element past a query's nb_q is written."""
+    wl = C.shrink(C.get("prefill"), [700, 2900, 33], new_tokens=37, page_perm=True, k_top=64)
+    cache, dec, st = run_step(wl, k=64)
+    assert st == 0
+    nq = wl.nq
+    inp = H.step_inputs(wl)
+    nb = ((inp["q_pos"].long() + 1) // 4).cpu()
+    width = int(nb.max()) + 40
+    ref = dec.scores[:nq, :int(nb.max())].cpu()
+    for ld, offset in [(width - width % 4, 0), (width - width % 4 + 3, 0), (width - width % 4, 1)]:
+        flat = torch.full((nq * ld + 8,), float("nan"), dtype=torch.float32, device="cuda")
+        scores = flat[offset:offset + nq * ld].view(nq, ld)
+        status = _status()
+        qsa.qsa_index_scores(cache, inp["q_idx"], inp["w"], inp["q_seq"], inp["q_pos"], scores, status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        got = scores.cpu()
+        for row in range(nq):
+            n = int(nb[row])
+            assert torch.equal(got[row, :n].view(torch.int32), ref[row, :n].view(torch.int32)), (ld, offset, row)
+            assert torch.isnan(got[row, n:]).all(), f"ld {ld} offset {offset}: row {row} written past nb_q"
+
+
 def test_topk_all_ties_take_lowest_indices():
     wl = C.shrink(C.get("quarter"), [2000], k_top=100)
     cache = H.new_cache(wl)
