@@ -12,6 +12,9 @@
 // 4 KiB kc pages (16 blocks x 128 dims): every lane issues 16-byte loads that
 // land directly in mma.sync m16n8k16 A fragments (rows = the page's 16
 // blocks, K = 128 dims, N = the 8 indexer heads), index_page.cuh.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "index_page.cuh"
 
 namespace {
@@ -131,16 +134,9 @@ struct TiledArgs {
   int64_t ld;
   int32_t bulk;  // score rows 16-byte aligned (base and pitch): scores leave by bulk copies
   int32_t* st;
+  CUtensorMap tm_kc;  // kc_pages as [num_pages * 16 rows][128 dims], boxes of 16 rows x 64 dims, 128-B swizzle
+  CUtensorMap tm_q;   // q_idx as [nq * 8 rows][128 dims], boxes of 256 rows x 64 dims, 128-B swizzle
 };
-
-__device__ __forceinline__ void cp_async16_cg(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 // ---------------------------------------------------------------------------
 // The contraction runs on the 5th-generation tensor cores (tcgen05): per
@@ -153,26 +149,27 @@ __device__ __forceinline__ void cp_async_wait_group() {
 //              quadrant a warp may access) and the columns of queries
 //              16 (w / 4) .. + 15, sums the heads, stages the scores in shared
 //              memory and stores each query's 32 consecutive scores with one
-//              128-byte bulk copy (cp.async.bulk, no multicast; element stores
+//              128-byte bulk copy (cp.async.bulk from this CTA; element stores
 //              when the caller's score rows are not 16-byte aligned)
 //   warp 8     TMEM allocation (512 columns: two accumulator buffers) and the
 //              MMA issue (one elected thread), tcgen05.commit to mbarriers
-//   warps 9-12 producers: 16-byte cp.async of q_idx (once) and of every kc
-//              tile into the canonical K-major, no-swizzle operand layout
-//              (8-row x 16-byte core matrices; the two 8-element halves of a
-//              16-element K step 128 B apart, 8-row groups 256 B apart), then
-//              a proxy fence and an mbarrier arrival per tile (a tile is
-//              published once the copies of the tile two later are issued,
-//              so three tiles are in flight per thread; 4-stage ring)
+//   warp 9     producer: tensor-map copies (one thread issues them) into the
+//              K-major 128-byte-swizzled operand layout (8-row x 128-byte
+//              atoms 1 KiB apart; dims 64 .. 127 one operand-height further):
+//              the q_idx operand once, then per kc tile its 8 pages x 2 halves
+//              of 16 rows x 64 dims, completing on the stage mbarrier by byte
+//              count (4-stage ring).  Each tile's page ids are loaded while the
+//              tile before it is copied.  Tensor-map copies move a tile with 16
+//              requests where 16-byte copies needed 2,048, which had capped the
+//              tile rate at about 19 GB/s per SM.
 // All waits are bounded; on expiry the CTA records QSA_DEV_TIMEOUT, stops
 // issuing work, drains what it issued and frees its tensor memory.
 
 constexpr int kUStages = 4;
 constexpr int kUTileBytes = kTB * kIdxDim * 2;                 // 32 KiB: one operand of 128 rows
-constexpr int kUEpiWarps = 8, kUMmaWarp = 8, kUProdWarp0 = 9, kUProdWarps = 4;
-constexpr int kUThreads = (kUProdWarp0 + kUProdWarps) * 32;    // 416
+constexpr int kUEpiWarps = 8, kUMmaWarp = 8, kUProdWarp0 = 9, kUProdWarps = 1;
+constexpr int kUThreads = (kUProdWarp0 + kUProdWarps) * 32;    // 320
 constexpr int kUEpiQ = kTQ * 4 / kUEpiWarps;                    // queries per epilogue warp: 16
-constexpr int kUProdThreads = kUProdWarps * 32;
 constexpr int kUN = kTQ * kIdxHeads;                           // 256: MMA N = the CTA's queries x heads
 constexpr int kUBBytes = kUN * kIdxDim * 2;                    // 64 KiB: the q_idx operand
 constexpr int kUAcc = 2;                                       // accumulator buffers in tensor memory
@@ -185,27 +182,36 @@ constexpr int kUOffBar = (kUOffMeta + (3 * kTQ + 4) * 4 + 7) & ~7;
 constexpr int kUNumBars = 2 * kUStages + 2 * kUAcc + 2;        // full/empty per stage, acc full/empty, b_full, done
 constexpr int kUStageFloats = kUEpiQ * 32;                     // one epilogue warp's 32 rows x 16 queries
 constexpr int kUOffStage = (kUOffBar + kUNumBars * 8 + 127) & ~127;  // 2 x 4 warps score staging buffers
-constexpr int kUSmem = kUOffStage + 2 * kUEpiWarps * kUStageFloats * 4;
+constexpr int kUSmem = kUOffStage + 2 * kUEpiWarps * kUStageFloats * 4 + 1024;  // + room to align the base to 1 KiB
 constexpr uint32_t kUIdesc = (1u << 4)                       // D: fp32
                            | (1u << 7) | (1u << 10)          // A, B: bf16
                            | ((uint32_t)(kUN >> 3) << 17)    // N = 256
                            | ((uint32_t)(128 >> 4) << 24);   // M = 128
 constexpr uint64_t kUWaitNs = 2000000000ull;
 
-// byte offset of 16-byte chunk c (dims 8c .. 8c+7) of row r of a `rows`-row operand
-template <int rows>
-__device__ __forceinline__ uint32_t umma_off(int r, int c) {
-  return (uint32_t)((c >> 1) * (rows * 32) + (r >> 3) * 256 + (c & 1) * 128 + (r & 7) * 16);
-}
-
-// shared-memory matrix descriptor: K-major, no swizzle, LBO 128 B, SBO 256 B
-__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
+// shared-memory matrix descriptor: K-major, 128-byte swizzle (8 rows x 128 B atoms, 1 KiB apart)
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)(128u >> 4) << 16;
-  d |= (uint64_t)(256u >> 4) << 32;
-  d |= (uint64_t)1u << 46;  // descriptor version for sm_100
+  d |= (uint64_t)(16u >> 4) << 16;     // leading byte offset: unused by this layout
+  d |= (uint64_t)(1024u >> 4) << 32;   // stride byte offset: between 8-row groups
+  d |= (uint64_t)1u << 46;             // descriptor version for sm_100
+  d |= (uint64_t)2u << 61;             // 128-byte swizzle
   return d;
+}
+// descriptor advance for 16-element K step ks of a `rows`-row operand: 64-dim halves
+// `rows` x 128 B apart, 32 B per step inside a half (in 16-byte units)
+template <int rows>
+__device__ __forceinline__ uint64_t ksteps(int ks) {
+  return (uint64_t)(((ks >> 2) * rows * 128 + (ks & 3) * 32) >> 4);
+}
+
+// 2-D tensor-map copy into this CTA's shared memory, completing on an mbarrier
+__device__ __forceinline__ void tma2d(uint32_t sdst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(sdst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
 }
 
 __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
@@ -260,10 +266,10 @@ __device__ __forceinline__ bool uwait(uint32_t bar, uint32_t parity, volatile in
   }
 }
 
-__global__ void __launch_bounds__(kUThreads, 1) index_scores_umma_kernel(TiledArgs a) {
+__global__ void __launch_bounds__(kUThreads, 1) index_scores_umma_kernel(const __grid_constant__ TiledArgs a) {
   pdl_launch_dependents();
   extern __shared__ __align__(128) uint8_t usmem[];
-  uint8_t* smem = usmem;
+  uint8_t* smem = usmem + (((smem_u32(usmem) + 1023u) & ~1023u) - smem_u32(usmem));  // 1 KiB aligned
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int32_t* t_seq = reinterpret_cast<int32_t*>(smem + kUOffMeta);
   int32_t* t_nb = t_seq + kTQ;
@@ -282,14 +288,14 @@ __global__ void __launch_bounds__(kUThreads, 1) index_scores_umma_kernel(TiledAr
 
   if (tid == 0) {
     for (int i = 0; i < kUStages; ++i) {
-      mbar_init(bar_full + i * 8, kUProdThreads);
+      mbar_init(bar_full + i * 8, 1);  // the producer's arrive with the tile's byte count
       mbar_init(bar_empty + i * 8, 1);
     }
     for (int i = 0; i < kUAcc; ++i) {
       mbar_init(bar_accf + i * 8, 1);
       mbar_init(bar_acce + i * 8, kUEpiWarps * 32);
     }
-    mbar_init(bar_bfull, kUProdThreads);
+    mbar_init(bar_bfull, 1);
     mbar_init(bar_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -355,85 +361,69 @@ __global__ void __launch_bounds__(kUThreads, 1) index_scores_umma_kernel(TiledAr
   };
 
   if (warp >= kUProdWarp0) {
-    // ---------------- producers
-    const int pt = tid - kUProdWarp0 * 32;  // 0..127
-    // q_idx operand: row = query * 8 + head, 16 chunks of 16 B
-    for (int e = pt; e < kTQ * kIdxHeads * 16; e += kUProdThreads) {
-      const int r = e >> 4, c = e & 15;
-      const int q = q0 + (r >> 3);
-      const uint32_t dst = sb + kUOffB + umma_off<kUN>(r, c);
-      if (q < a.nq)
-        cp_async16_cg(dst, a.q_idx + ((size_t)q * kIdxHeads + (r & 7)) * kIdxDim + c * 8);
-      else
-        sts128(dst, make_uint4(0, 0, 0, 0));
+    // ---------------- producer warp: tensor-map copies, issued by lane 0.  The q_idx
+    // operand (two 256-row x 64-dim boxes; rows past nq * 8 read as zero) once, then
+    // per kc tile 8 pages x 2 halves of 16 rows x 64 dims.  A tile's page ids are
+    // loaded (lane p: page p) while the tile before it is copied; a rejected page
+    // reads rows past the tensor, which arrive as zeros.
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_bfull, (uint32_t)kUBBytes);
+      tma2d(sb + kUOffB, &a.tm_q, 0, q0 * kIdxHeads, bar_bfull);
+      tma2d(sb + kUOffB + kUN * 128, &a.tm_q, 64, q0 * kIdxHeads, bar_bfull);
     }
-    cp_async_commit();
-    cp_async_wait_group<0>();
-    fence_async_smem();
-    mbar_arrive(bar_bfull);
-    int j = 0;  // global tile counter
-    int pend0 = -1, pend1 = -1;  // tiles whose copies are in flight and not yet signalled (older first)
+    int j = 0;
     for (int si = 0; si < nseq && !*abort_flag; ++si) {
       int64_t B0, B1;
       pass_range(si, B0, B1);
       const int S = t_list[si];
-      // warp w copies chunks 4w .. 4w+3 of every row; lane l takes row 8k + (l & 7),
-      // chunk 4w + (l >> 3): one warp instruction writes 8 rows x 4 chunks, which the
-      // canonical layout puts in 4 lines of 8 distinct 16-byte bank groups (the
-      // minimum 4 wavefronts for 512 B), and reads 8 x 64 contiguous bytes.  A tile's
-      // page ids are loaded while the tile before it is copied, so no tile waits for
-      // a page-table round trip before its copies are issued.
-      constexpr int kPer = kTB * 16 / kUProdThreads;  // 16
-      const int c = 4 * (pt >> 5) + ((pt & 31) >> 3);
-      auto load_ids = [&](int64_t tb0, int (&ph)[kPer]) {
-#pragma unroll
-        for (int k = 0; k < kPer; ++k) {
-          const int64_t b = tb0 + 8 * k + (pt & 7);
-          ph[k] = b < B1 ? __ldg(a.bt + (int64_t)S * a.mpps + b / kBlocksPerPage) : -1;
-        }
+      auto load_ids = [&](int64_t tb0) {
+        const int64_t bp = tb0 + (int64_t)kBlocksPerPage * lane;
+        return (lane < kTB / kBlocksPerPage && bp < B1) ? __ldg(a.bt + (int64_t)S * a.mpps + bp / kBlocksPerPage) : -1;
       };
-      int phys[kPer];
-      load_ids(B0, phys);
+      int phys = load_ids(B0);
+      bool ok_all = true;
       for (int64_t b0 = B0; b0 < B1; b0 += kTB, ++j) {
         const int stage = j % kUStages;
-        if (j >= kUStages && !uwait(bar_empty + stage * 8, (uint32_t)((j / kUStages - 1) & 1), abort_flag, a.st))
+        int okw = 1;
+        if (lane == 0 && j >= kUStages)
+          okw = uwait(bar_empty + stage * 8, (uint32_t)((j / kUStages - 1) & 1), abort_flag, a.st) ? 1 : 0;
+        okw = __shfl_sync(0xffffffffu, okw, 0);
+        __syncwarp();
+        if (!okw) {
+          ok_all = false;
           break;
+        }
+        const int next = load_ids(b0 + kTB);
+        const bool good = phys >= 0 && phys < a.num_pages;
+        if (lane < kTB / kBlocksPerPage && !good && b0 + (int64_t)kBlocksPerPage * lane < B1) flag(a.st, QSA_DEV_BAD_PAGE);
+        const int y = good ? phys * kBlocksPerPage : a.num_pages * kBlocksPerPage;
         const uint32_t tile = sb + kUOffA + stage * kUTileBytes;
+        if (lane == 0) mbar_arrive_expect_tx(bar_full + stage * 8, (uint32_t)kUTileBytes);
 #pragma unroll
-        for (int k = 0; k < kPer; ++k) {
-          const int r = 8 * k + (pt & 7);
-          const int64_t b = b0 + r;
-          const uint32_t dst = tile + umma_off<kTB>(r, c);
-          if (b < B1 && phys[k] >= 0 && phys[k] < a.num_pages) {
-            cp_async16_cg(dst, a.kc + ((size_t)phys[k] * kBlocksPerPage + b % kBlocksPerPage) * kIdxDim + c * 8);
-          } else {
-            sts128(dst, make_uint4(0, 0, 0, 0));
-            if (b < B1 && c == 0) flag(a.st, QSA_DEV_BAD_PAGE);
+        for (int p = 0; p < kTB / kBlocksPerPage; ++p) {
+          const int yp = __shfl_sync(0xffffffffu, y, p);
+          if (lane == 0) {
+            tma2d(tile + p * kBlocksPerPage * 128, &a.tm_kc, 0, yp, bar_full + stage * 8);
+            tma2d(tile + kTB * 128 + p * kBlocksPerPage * 128, &a.tm_kc, 64, yp, bar_full + stage * 8);
           }
         }
-        cp_async_commit();
-        int next[kPer];  // the next tile's page ids, in flight during the waits below
-        load_ids(b0 + kTB, next);
-        if (pend0 >= 0) {  // the copies of the tile issued two tiles ago have landed: publish it
-          cp_async_wait_group<2>();
-          fence_async_smem();
-          mbar_arrive(bar_full + (pend0 % kUStages) * 8);
-        }
-        pend0 = pend1;
-        pend1 = j;
-#pragma unroll
-        for (int k = 0; k < kPer; ++k) phys[k] = next[k];
+        phys = next;
       }
+      if (!ok_all) break;
     }
-    cp_async_wait_group<0>();
-    fence_async_smem();
-    if (pend0 >= 0) mbar_arrive(bar_full + (pend0 % kUStages) * 8);
-    if (pend1 >= 0) mbar_arrive(bar_full + (pend1 % kUStages) * 8);
+    // every copy this warp issued has landed before the CTA moves on (the last
+    // tile of each stage and the q_idx operand; bounded, as every wait here)
+    if (lane == 0) {
+      (void)mbar_wait_bounded(bar_bfull, 0, kUWaitNs);
+      for (int t = j - kUStages < 0 ? 0 : j - kUStages; t < j; ++t)
+        (void)mbar_wait_bounded(bar_full + (t % kUStages) * 8, (uint32_t)((t / kUStages) & 1), kUWaitNs);
+    }
+    __syncwarp();
   } else if (warp == kUMmaWarp) {
     // ---------------- MMA issue (one thread)
     if (lane == 0) {
       bool ok = uwait(bar_bfull, 0, abort_flag, a.st);
-      const uint64_t bdesc0 = umma_desc(sb + kUOffB);
+      const uint64_t bdesc0 = umma_desc_sw128(sb + kUOffB);
       int j = 0;
       for (int si = 0; si < nseq && ok; ++si) {
         int64_t B0, B1;
@@ -446,11 +436,10 @@ __global__ void __launch_bounds__(kUThreads, 1) index_scores_umma_kernel(TiledAr
             break;
           }
           tc_fence_after();
-          const uint64_t adesc0 = umma_desc(sb + kUOffA + stage * kUTileBytes);
+          const uint64_t adesc0 = umma_desc_sw128(sb + kUOffA + stage * kUTileBytes);
 #pragma unroll
           for (int ks = 0; ks < kIdxDim / 16; ++ks)  // per 16-element K step: rows * 32 B, in 16-B units
-            umma_f16(tmem + acc * kUN, adesc0 + (uint64_t)(ks * kTB * 2), bdesc0 + (uint64_t)(ks * kUN * 2), kUIdesc,
-                     ks > 0 ? 1u : 0u);
+            umma_f16(tmem + acc * kUN, adesc0 + ksteps<kTB>(ks), bdesc0 + ksteps<kUN>(ks), kUIdesc, ks > 0 ? 1u : 0u);
           umma_commit(bar_empty + stage * 8);  // the kc stage is free once these MMAs finish
           umma_commit(bar_accf + acc * 8);     // the accumulator is ready
         }
@@ -549,6 +538,36 @@ __global__ void __launch_bounds__(kUThreads, 1) index_scores_umma_kernel(TiledAr
 
 bool aligned(const void* p, unsigned a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+// The two tensor maps of the query-tiled kernel (the driver's encoder is looked
+// up once through the runtime).  Both views are [rows][128 dims] BF16 with rows
+// 256 B apart; boxes of 64 dims (128 B, the swizzle span) by 16 rows (one kc
+// page) or 256 rows (the 32 queries x 8 heads of a CTA).
+bool encode_maps(TiledArgs& t, const void* kc, int32_t num_pages, const void* q_idx, int32_t nq) {
+  static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  if (!enc) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !f) {
+      (void)cudaGetLastError();
+      return false;
+    }
+    enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  const cuuint64_t strides[1] = {(cuuint64_t)kIdxDim * 2};
+  const cuuint32_t es[2] = {1, 1};
+  const cuuint64_t kdims[2] = {(cuuint64_t)kIdxDim, (cuuint64_t)num_pages * kBlocksPerPage};
+  const cuuint32_t kbox[2] = {64, (cuuint32_t)kBlocksPerPage};
+  const cuuint64_t qdims[2] = {(cuuint64_t)kIdxDim, (cuuint64_t)nq * kIdxHeads};
+  const cuuint32_t qbox[2] = {64, (cuuint32_t)kUN};
+  return enc(&t.tm_kc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kc), kdims, strides, kbox, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS &&
+         enc(&t.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q_idx), qdims, strides, qbox, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 extern "C" int qsa_index_scores(const qsa_cache_t* cache, const void* q_idx, const float* w, const int32_t* q_seq,
@@ -572,8 +591,11 @@ extern "C" int qsa_index_scores(const qsa_cache_t* cache, const void* q_idx, con
   a.q_pos = q_pos;
   a.scores = scores;
   a.ld = scores_ld;
-  // Many queries per sequence (chunked prefill): the query-tiled contraction.
-  if ((int64_t)nq >= 8 * (int64_t)cache->max_seqs && nq >= kTQ) {
+  // Many queries per sequence (chunked prefill): the query-tiled contraction,
+  // while every row coordinate of its tensor maps fits 32 bits.
+  const bool coords_fit = (int64_t)cache->num_pages * kBlocksPerPage + kBlocksPerPage <= 0x7fffffff &&
+                          (int64_t)nq * kIdxHeads + kUN <= 0x7fffffff;
+  if ((int64_t)nq >= 8 * (int64_t)cache->max_seqs && nq >= kTQ && coords_fit) {
     TiledArgs t;
     t.kc = static_cast<const __nv_bfloat16*>(cache->kc_pages);
     t.bt = cache->block_table;
@@ -594,6 +616,7 @@ extern "C" int qsa_index_scores(const qsa_cache_t* cache, const void* q_idx, con
     const int64_t gy = (max_blocks + kTChunkBlocks - 1) / kTChunkBlocks;
     const int64_t gx = ((int64_t)nq + kTQ - 1) / kTQ;
     if (gy > 65535 || gx > 0x7fffffff) return QSA_ERR_UNSUPPORTED;
+    if (!encode_maps(t, cache->kc_pages, cache->num_pages, q_idx, nq)) return QSA_ERR_CUDA;
     if (cudaFuncSetAttribute(index_scores_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kUSmem) !=
         cudaSuccess) {
       (void)cudaGetLastError();
