@@ -105,6 +105,11 @@ __device__ __forceinline__ void st_cluster(void* p, uint32_t rank, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(remote), "r"(v) : "memory");
 }
 
+// Bulk prefetch of `bytes` (a multiple of 16, 16-byte aligned) into L2.
+__device__ __forceinline__ void l2_prefetch_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 __global__ void __launch_bounds__(kFThreads, 2) index_topk_kernel(FusedArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   FSmem& S = *reinterpret_cast<FSmem*>(smem_raw);
@@ -172,6 +177,15 @@ __global__ void __launch_bounds__(kFThreads, 2) index_topk_kernel(FusedArgs a) {
         const int phys = pl < np_cta ? ids[pl] : -1;
         ok[k] = pl < np_cta && phys >= 0 && phys < a.num_pages;
         if (ok[k]) load_idx_page(a.kc, phys, ra[k], rb[k]);
+      }
+      // the warp's next two pages go to L2 now (lanes 0 and 1, one bulk
+      // prefetch of 4 KiB each): the next loads find them there, and the
+      // bytes in flight per SM are no longer bounded by these registers
+      if (lane < 2) {
+        const int pn = pp + 2 * kFWarps + lane;
+        const int phys = pn < np_cta ? ids[pn] : -1;
+        if (phys >= 0 && phys < a.num_pages)
+          l2_prefetch_bulk(a.kc + (size_t)phys * kBlocksPerPage * kIdxDim, kBlocksPerPage * kIdxDim * 2);
       }
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
